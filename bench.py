@@ -1,0 +1,437 @@
+#!/usr/bin/env python
+"""Benchmark of the entropy-bound canvas sampler step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: one 256 x 262144 bf16 canvas per GPU (the model card's canvas and
+vocabulary), seeded synthetic decoder logits pre-generated for all 48 steps of
+an entropy-bound trajectory (temperature 0.8 -> 0.4, entropy_bound 0.1,
+adaptive stop 0.005 / 1 stable step).  A "step" is one eb_sampler_step call:
+every logit of every active canvas read once, entropies, argmax, draws,
+commit, renoise, stop test.  Each step reads its own 134 MB of logits, more
+than the 126 MB L2, so no step hits in L2 on the previous one's data.
+
+Timing: W eager warm-up steps, then exactly K steps timed with CUDA events on
+the launching stream between a barrier + synchronize on both sides (max over
+ranks); full 48-step trajectories are replayed from one CUDA graph, the
+remainder runs eagerly.  The kernel's own launch durations (for the roofline)
+come from per-launch events over one eager trajectory.  For N > 1 each rank
+runs its own canvas (global canvas index = rank): no data-path collective,
+weak scaling.
+
+--impl reference times the CPU oracle (the float64 restatement in oracle/)
+on the host cores, rank 0 only, on bounded samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "canvas positions sampled/sec and HBM GB/s (% of B200 peak), 256x262144 bf16 step"
+UNIT = "positions/s"
+WORKLOAD = "canvas"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=9600)
+    p.add_argument("--warmup", type=int, default=48)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--e2e-steps", type=int, default=48)
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("eb_step.cuh", "eb_device.cuh", "eb_sampler.cu"):
+        with open(os.path.join(ROOT, "entropy_bound_canvas_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the step kernel from the committed ncu summary,
+    if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "step_kernel_canvas_1x256x262144_bf16.md")
+    try:
+        txt = open(path).read()
+    except OSError:
+        return None
+    m1 = re.search(r"source_sha256_16:\s*([0-9a-f]{16})", txt)
+    m2 = re.search(r"dram_bytes_per_launch:\s*([0-9]+)", txt)
+    if not m1 or not m2 or m1.group(1) != kernel_source_hash():
+        return None
+    return int(m2.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        sm, smax, reasons, power = [], None, set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+                power.append(float(f[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [x for x, p in zip(sm, power) if p > 200.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle as O
+    import synth
+
+    w = synth.WORKLOADS[WORKLOAD]
+    cfg = O.Config(B=w.B, L=w.L, V=w.V, group_size=64, **w.sampler_config())
+    # Per step: the oracle's full per-position work (entropy, argmax, two-level
+    # draw) on ROWS positions of the canvas at that step, plus the canvas
+    # decisions; bounded so the whole run ends within a few minutes.
+    rows_per_step = 4
+    K, W = args.steps, args.warmup
+    total = K + W
+    budget_rows = 12000  # ~2 minutes of rows at ~10 ms each
+    if total * rows_per_step > budget_rows:
+        rows_per_step = max(1, budget_rows // total)
+    st = O.State(cfg).init()
+    times = []
+    for i in range(total):
+        s = i % w.num_steps
+        l0 = (i * 37) % (w.L - rows_per_step + 1)
+        rows = synth.generate_host(w, s, 0, 1, l0, rows_per_step)[0]
+        t0 = time.perf_counter()
+        T = O.temperature(cfg, s)
+        H = np.zeros(w.L)
+        amax = np.zeros(w.L, np.int32)
+        pm = np.zeros(w.L)
+        smp = np.zeros(w.L, np.int32)
+        for k in range(rows_per_step):
+            l = l0 + k
+            H[l], pm[l], amax[l], _ = O.row_stats(rows[k], 1.0 / T)
+            if not st.committed[0, l]:
+                smp[l] = O.sample(cfg, rows[k], 1.0 / T, 0, l, s)[0]
+        O.canvas_decide(st, 0, s, H, amax, pm, smp)
+        dt = time.perf_counter() - t0
+        if st.stop[0] or s == w.num_steps - 1:
+            st = O.State(cfg).init()
+        if i >= W:
+            times.append(dt)
+    el = sum(times)
+    value = K * rows_per_step / el
+    sample = (f"{rows_per_step} of 256 positions per step (entropy, argmax and two-level draw "
+              f"of each, 262144 bf16 logits) plus the canvas decisions; {K} timed steps")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": K, "warmup": W, "ms_per_step": 1e3 * el / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "canvas 1x256x262144 bf16 (oracle sample)", "B": 1, "L": 256,
+                   "V": 262144},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- our arm
+
+def cpu_baseline(w, logits_steps, states):
+    """The oracle, as it stands, on full canvas steps at a few step indices."""
+    import numpy as np
+
+    import oracle as O
+    cfg = O.Config(B=w.B, L=w.L, V=w.V, group_size=64, **w.sampler_config())
+    t_total, n_pos = 0.0, 0
+    used = []
+    for s, (cv, cm, prev) in states.items():
+        st = O.State(cfg).init()
+        st.canvas[0], st.committed[0], st.prev[0] = cv, cm, prev
+        lg = logits_steps[s][0].view(__import__("torch").int16).cpu().numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        O.step_canvas(st, 0, lg, s)
+        t_total += time.perf_counter() - t0
+        n_pos += w.L
+        used.append(s)
+    return {"value": n_pos / t_total, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"full 256-position canvas steps at s={used} of the same trajectory "
+                      f"(single thread, float64), {t_total:.1f} s of CPU work"}
+
+
+def run_ours(args):
+    import torch
+
+    import entropy_bound_canvas_b200 as E
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    w = synth.WORKLOADS[WORKLOAD]
+    N = w.num_steps
+    K, W = args.steps, max(3, args.warmup)
+    stream = torch.cuda.current_stream(dev)
+
+    # inputs resident in HBM: this rank's canvas for all N steps
+    logits = [torch.empty((w.B, w.L, w.V), dtype=torch.bfloat16, device=dev) for _ in range(N)]
+    for s in range(N):
+        synth.generate_device(w, s, logits[s], b0=rank)
+    eb = E.EBSampler(w.B, w.L, w.V, device=dev, canvas_offset=rank, **w.sampler_config())
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    torch.cuda.synchronize()
+
+    # reference trajectory (untimed): active canvases per step, snapshots for the CPU baseline
+    active = []
+    snaps = {}
+    eb.init_canvas(canvas, committed, stop)
+    for s in range(N):
+        active.append(int((stop == 0).sum().item()))
+        if s in (0, 12, 24, 36, 47):
+            snaps[s] = (canvas[0].cpu().numpy().copy(), committed[0].cpu().numpy().copy(),
+                        amax[0].cpu().numpy().copy())
+        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    stop_step = next((s for s in range(N) if s + 1 < N and active[s + 1] == 0), N - 1)
+
+    # warm-up: W eager steps along the trajectory
+    eb.init_canvas(canvas, committed, stop)
+    for i in range(W):
+        s = i % N
+        if s == 0 and i > 0:
+            eb.init_canvas(canvas, committed, stop)
+        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+
+    # one trajectory as a CUDA graph
+    g = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        eb.init_canvas(canvas, committed, stop)
+        for s in range(N):
+            eb.step(logits[s], s, canvas, committed, H, amax, stop)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            eb.init_canvas(canvas, committed, stop)
+            for s in range(N):
+                eb.step(logits[s], s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+
+    full, rem = divmod(K, N)
+    launches = full * (N + 1) + (rem + (1 if rem else 0))
+    pos_per_traj = sum(active) * w.L
+    positions = full * pos_per_traj + sum(active[:rem]) * w.L
+    bytes_steps = full * sum(active) + sum(active[:rem])
+    bytes_total = bytes_steps * w.L * w.V * 2
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(full):
+        g.replay()
+    if rem:
+        eb.init_canvas(canvas, committed, stop)
+        for s in range(rem):
+            eb.step(logits[s], s, canvas, committed, H, amax, stop)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    el_ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([el_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        el_ms = float(t.item())
+        p = torch.tensor([positions, bytes_total], device=dev, dtype=torch.float64)
+        dist.all_reduce(p, op=dist.ReduceOp.SUM)
+        positions_all, bytes_all = float(p[0].item()), float(p[1].item())
+    else:
+        positions_all, bytes_all = float(positions), float(bytes_total)
+    value = positions_all / (el_ms * 1e-3)
+    hbm_gbs_job = bytes_all / (el_ms * 1e-3) / 1e9
+
+    # per-launch kernel durations over one eager trajectory (for the roofline)
+    evs = []
+    eb.init_canvas(canvas, committed, stop)
+    for s in range(N):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+        b.record(stream)
+        evs.append((s, a, b))
+    torch.cuda.synchronize()
+    durs = [(s, a.elapsed_time(b)) for s, a, b in evs if active[s] and s > 0]
+    k_ms = statistics.mean(d for _, d in durs)
+    k_bytes = w.B * w.L * w.V * 2  # algorithmic: every logit of the active canvas once
+    achieved = k_bytes / (k_ms * 1e-3) / 1e9
+    peak, peak_kind = peaks()
+    traffic = recorded_traffic()
+
+    # end-to-end: host (pinned) logits -> device, step, result back to host, every step
+    e2e = None
+    if not args.no_e2e:
+        n_e2e = min(args.e2e_steps, N)
+        host = [logits[s].cpu().pin_memory() for s in range(n_e2e)]
+        dev_buf = torch.empty_like(logits[0])
+        out_cv = torch.empty((w.B, w.L), dtype=torch.int32).pin_memory()
+        out_cm = torch.empty((w.B, w.L), dtype=torch.uint8).pin_memory()
+        out_sp = torch.empty((w.B,), dtype=torch.uint8).pin_memory()
+        eb.init_canvas(canvas, committed, stop)
+        torch.cuda.synchronize()
+        barrier()
+        t0 = time.perf_counter()
+        x0, x1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        x0.record(stream)
+        pos_e2e = 0
+        for s in range(n_e2e):
+            dev_buf.copy_(host[s], non_blocking=True)
+            eb.step(dev_buf, s, canvas, committed, H, amax, stop)
+            out_cv.copy_(canvas, non_blocking=True)
+            out_cm.copy_(committed, non_blocking=True)
+            out_sp.copy_(stop, non_blocking=True)
+            stream.synchronize()
+            pos_e2e += active[s] * w.L
+        x1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = x0.elapsed_time(x1)
+        if dist is not None:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+            pos_e2e *= world
+        e2e = {"value": pos_e2e / (e2e_ms * 1e-3), "unit": UNIT,
+               "h2d_bytes_per_step": w.B * w.L * w.V * 2,
+               "d2h_bytes_per_step": w.B * w.L * 4 + w.B * w.L + w.B,
+               "steps": n_e2e, "wall_s": time.perf_counter() - t0}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, logits, snaps)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {
+                "workload": "canvas 1x256x262144 bf16 per GPU, 48-step entropy-bound trajectory",
+                "B_per_gpu": w.B, "L": w.L, "V": w.V, "num_steps": N, "seed": w.seed,
+                "stop_step": stop_step,
+                "l2": "inputs larger than L2: each step reads its own 134 MB of logits",
+                "timing": "full 48-step trajectories replayed from one CUDA graph, remainder eager",
+            },
+            "hbm_gbs": hbm_gbs_job,
+            "hbm_frac_of_peak": hbm_gbs_job / (peak * world),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "kernel": "ebk::step_kernel<bf16, bulk-copy>",
+                         "kernel_ms": k_ms, "algorithmic_bytes": k_bytes,
+                         "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    del g
+    eb.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

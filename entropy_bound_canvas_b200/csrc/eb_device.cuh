@@ -1,0 +1,156 @@
+// eb_device.cuh -- device primitives of the sampler: Philox4x32-10, the
+// Gumbel and uniform-token maps, mbarrier / bulk-copy (TMA) wrappers with
+// bounded waits, and warp reductions.  sm_100a only.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace ebk {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+// 2^x with the MUFU approximation (relative error ~2^-22); subnormal results
+// flush to zero, which only drops terms below 2^-126 of the row maximum.
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float lg2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// ---------------------------------------------------------------------------
+// Philox4x32-10 (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
+// SC'11): ten rounds of two 32x32->64 multiplies, the high halves crossed with
+// the other two words and the round key, the key bumped by the Weyl constants.
+// ---------------------------------------------------------------------------
+struct Words4 {
+  uint32_t w[4];
+};
+
+__device__ __forceinline__ Words4 philox(uint32_t c0, uint32_t c1, uint32_t c2, uint32_t c3,
+                                         uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    const uint32_t n0 = hi1 ^ c1 ^ k0;
+    const uint32_t n2 = hi0 ^ c3 ^ k1;
+    c0 = n0;
+    c1 = lo1;
+    c2 = n2;
+    c3 = lo0;
+  }
+  Words4 o;
+  o.w[0] = c0;
+  o.w[1] = c1;
+  o.w[2] = c2;
+  o.w[3] = c3;
+  return o;
+}
+
+__device__ __forceinline__ uint32_t pick_word(const Words4& r, uint32_t i) {
+  return i == 0 ? r.w[0] : i == 1 ? r.w[1] : i == 2 ? r.w[2] : r.w[3];
+}
+
+// Streams of the counter layout: ctr = (index >> 2, a, step, b | stream << 24).
+enum : uint32_t { kStreamGumbel = 0, kStreamRenoise = 1, kStreamInit = 2, kStreamGroup = 3 };
+
+// Standard Gumbel from one word: u = (2 (x >> 9) + 1) 2^-24 (exact in fp32),
+// g = -ln(-ln u).  The inner log must be accurate near u = 1 (logf, ~1 ulp);
+// the outer one only needs absolute accuracy, which lg2.approx gives.
+__device__ __forceinline__ float gumbel(uint32_t x) {
+  const float u = (float)((x >> 9) * 2u + 1u) * 5.9604644775390625e-08f;
+  const float e = -logf(u);
+  return -0.6931471805599453f * lg2(e);
+}
+
+// Largest Gumbel value the 23-bit grid can produce, -ln(-ln(1 - 2^-24)) =
+// 16.6355..., rounded up; a group whose log-partition plus this bound is
+// below the best score so far cannot win.
+constexpr float kGumbelMax = 16.64f;
+
+// Uniform token in [0, V): high word of x * V.
+__device__ __forceinline__ uint32_t uniform_token(uint32_t x, uint32_t V) { return __umulhi(x, V); }
+
+// ---------------------------------------------------------------------------
+// mbarrier + 1-D bulk copy (cp.async.bulk, the TMA engine without a tensor
+// map).  No multicast anywhere: every copy reads this GPU's own memory into
+// this CTA's shared memory.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Every wait on a barrier gives up after this long and reports a timeout.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::
+          "r"(smem_u32(smem_dst)),
+      "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Named barrier among the consumer warps only (the producer warp never joins).
+__device__ __forceinline__ void consumer_sync(int nthreads) {
+  asm volatile("bar.sync 1, %0;" ::"r"(nthreads) : "memory");
+}
+
+}  // namespace ebk

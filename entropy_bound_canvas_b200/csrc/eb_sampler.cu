@@ -1,0 +1,421 @@
+// eb_sampler.cu -- host side of the C ABI declared in include/eb_sampler.h.
+//
+// Validation, the device workspace, launch configuration (one persistent
+// step kernel per call, sized to fill every SM) and error codes.  All the
+// per-step arithmetic runs in the kernels of eb_step.cuh.
+#include "eb_sampler.h"
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <new>
+
+#include "eb_step.cuh"
+
+namespace {
+
+using ebk::Partial;
+using ebk::StepArgs;
+
+struct KernelCfg {
+  const void* fn = nullptr;
+  size_t smem = 0;
+  int grid = 0;
+};
+
+}  // namespace
+
+struct eb_sampler {
+  eb_config_t cfg;
+  int device = 0;
+  int sms = 0;
+  int ng = 0;
+  int max_segs = 0;
+  KernelCfg k[2][2];  // [dtype][tma]
+  // workspace (one allocation)
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  Partial* partials = nullptr;
+  uint32_t* row_ticket = nullptr;
+  uint32_t* canvas_ticket = nullptr;
+  uint32_t* exit_ticket = nullptr;
+  uint32_t* status = nullptr;
+  int32_t* prev_amax = nullptr;
+  int32_t* stable = nullptr;
+  int32_t* sample = nullptr;
+  float* pmax = nullptr;
+  uint8_t* stop_next = nullptr;
+  size_t tickets_bytes = 0;  // row + canvas + exit tickets, contiguous
+  int last_step = -1;
+};
+
+namespace {
+
+// Restores the caller's current device on scope exit.
+struct DeviceGuard {
+  int prev = -1;
+  bool ok = false;
+  explicit DeviceGuard(int dev) {
+    if (cudaGetDevice(&prev) == cudaSuccess && cudaSetDevice(dev) == cudaSuccess) ok = true;
+  }
+  ~DeviceGuard() {
+    if (prev >= 0) cudaSetDevice(prev);
+  }
+};
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+int validate_config(const eb_config_t* c) {
+  if (!c) return EB_ERR_INVALID_ARG;
+  if (c->B < 1 || c->L < 1 || c->V < 1 || c->num_steps < 1) return EB_ERR_INVALID_ARG;
+  if (c->B > EB_MAX_CANVASES || c->L > EB_MAX_POSITIONS) return EB_ERR_OVERFLOW;
+  if (c->canvas_offset < 0 || (int64_t)c->canvas_offset + c->B > (int64_t)(1 << 24))
+    return EB_ERR_OVERFLOW;
+  if (c->rule != EB_RULE_ENTROPY_BOUND && c->rule != EB_RULE_BLOCK_REFINEMENT &&
+      c->rule != EB_RULE_ENTROPY_BOUND_MI)
+    return EB_ERR_INVALID_ARG;
+  if (c->greedy != 0 && c->greedy != 1) return EB_ERR_INVALID_ARG;
+  if (!c->greedy && !(c->t_max > 0.0 && c->t_min > 0.0 && std::isfinite(c->t_max) &&
+                      std::isfinite(c->t_min)))
+    return EB_ERR_INVALID_ARG;
+  if (!(c->entropy_bound >= 0.0) || !std::isfinite(c->entropy_bound)) return EB_ERR_INVALID_ARG;
+  if (std::isnan(c->stop_entropy) || std::isnan(c->threshold)) return EB_ERR_INVALID_ARG;
+  if (c->stability_steps < 0 || c->quota < 0) return EB_ERR_INVALID_ARG;
+  // group numbering fits the 64-bit work split: B * L * ng * grid < 2^63
+  const uint64_t ng = ((uint64_t)c->V + ebk::kGroup - 1) / ebk::kGroup;
+  if ((uint64_t)c->B * (uint64_t)c->L * ng >= (1ull << 46)) return EB_ERR_OVERFLOW;
+  return EB_OK;
+}
+
+template <int DT, bool TMA>
+int setup_kernel(eb_sampler* h, const cudaDeviceProp& prop) {
+  KernelCfg& kc = h->k[DT][TMA ? 1 : 0];
+  const ebk::Layout lay = ebk::make_layout(DT, h->cfg.B, h->cfg.L);
+  kc.fn = reinterpret_cast<const void*>(&ebk::step_kernel<DT, TMA>);
+  kc.smem = lay.total;
+  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
+  if (cudaFuncSetAttribute(ebk::step_kernel<DT, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kc.smem) != cudaSuccess)
+    return EB_ERR_CUDA;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::step_kernel<DT, TMA>,
+                                                    ebk::kThreads, kc.smem) != cudaSuccess ||
+      per_sm < 1)
+    return EB_ERR_CUDA;
+  const uint64_t groups = (uint64_t)h->cfg.B * (uint64_t)h->cfg.L * (uint64_t)h->ng;
+  const uint64_t want = (groups + ebk::kTileGroups - 1) / ebk::kTileGroups;
+  kc.grid = (int)std::min<uint64_t>((uint64_t)per_sm * (uint64_t)prop.multiProcessorCount,
+                                    std::max<uint64_t>(1, want));
+  return EB_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V) {
+  if (!cfg) return;
+  std::memset(cfg, 0, sizeof(*cfg));
+  cfg->B = B;
+  cfg->L = L;
+  cfg->V = V;
+  cfg->num_steps = 48;
+  cfg->t_max = 0.8;
+  cfg->t_min = 0.4;
+  cfg->entropy_bound = 0.1;
+  cfg->stop_entropy = 0.005;
+  cfg->stability_steps = 1;
+  cfg->rule = EB_RULE_ENTROPY_BOUND;
+  cfg->threshold = 0.9;
+  cfg->quota = (L + 47) / 48;
+  cfg->greedy = 0;
+  cfg->canvas_offset = 0;
+  cfg->seed = 0;
+}
+
+int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
+  if (!out) return EB_ERR_INVALID_ARG;
+  *out = nullptr;
+  int rc = validate_config(cfg);
+  if (rc != EB_OK) return rc;
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess) return EB_ERR_CUDA;
+  if (device < 0 || device >= ndev) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaDeviceProp prop;
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return EB_ERR_CUDA;
+  if (prop.major != 10) return EB_ERR_UNSUPPORTED;
+
+  eb_sampler* h = new (std::nothrow) eb_sampler();
+  if (!h) return EB_ERR_OUT_OF_MEMORY;
+  h->cfg = *cfg;
+  h->device = device;
+  h->sms = prop.multiProcessorCount;
+  h->ng = (int)(((int64_t)cfg->V + ebk::kGroup - 1) / ebk::kGroup);
+
+  if ((rc = setup_kernel<ebk::kF32, true>(h, prop)) != EB_OK ||
+      (rc = setup_kernel<ebk::kF32, false>(h, prop)) != EB_OK ||
+      (rc = setup_kernel<ebk::kBF16, true>(h, prop)) != EB_OK ||
+      (rc = setup_kernel<ebk::kBF16, false>(h, prop)) != EB_OK) {
+    delete h;
+    return rc;
+  }
+  // Most CTAs one row can span: with one active canvas each CTA owns at
+  // least floor(L ng / G) groups, so a row meets at most
+  // floor((ng - 1) G / (L ng)) + 2 of them.
+  int gmax = 0;
+  for (int d = 0; d < 2; ++d)
+    for (int t = 0; t < 2; ++t) gmax = std::max(gmax, h->k[d][t].grid);
+  const uint64_t Lng = (uint64_t)cfg->L * (uint64_t)h->ng;
+  const uint64_t segs = ((uint64_t)(h->ng - 1) * (uint64_t)gmax) / Lng + 2;
+  h->max_segs = (int)std::min<uint64_t>((uint64_t)gmax, segs);
+
+  const size_t BL = (size_t)cfg->B * (size_t)cfg->L;
+  size_t off = 0;
+  const size_t o_part = off;
+  off = align256(off + sizeof(Partial) * BL * (size_t)h->max_segs);
+  const size_t o_tick = off;
+  h->tickets_bytes = sizeof(uint32_t) * (BL + (size_t)cfg->B + 1);
+  off = align256(off + h->tickets_bytes);
+  const size_t o_status = off;
+  off = align256(off + sizeof(uint32_t));
+  const size_t o_prev = off;
+  off = align256(off + sizeof(int32_t) * BL);
+  const size_t o_stable = off;
+  off = align256(off + sizeof(int32_t) * (size_t)cfg->B);
+  const size_t o_sample = off;
+  off = align256(off + sizeof(int32_t) * BL);
+  const size_t o_pmax = off;
+  off = align256(off + sizeof(float) * BL);
+  const size_t o_stopn = off;
+  off = align256(off + (size_t)cfg->B);
+  h->ws_bytes = off;
+  if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
+    cudaGetLastError();
+    delete h;
+    return EB_ERR_OUT_OF_MEMORY;
+  }
+  if (cudaMemset(h->ws, 0, h->ws_bytes) != cudaSuccess) {
+    cudaFree(h->ws);
+    delete h;
+    return EB_ERR_CUDA;
+  }
+  char* base = static_cast<char*>(h->ws);
+  h->partials = reinterpret_cast<Partial*>(base + o_part);
+  h->row_ticket = reinterpret_cast<uint32_t*>(base + o_tick);
+  h->canvas_ticket = h->row_ticket + BL;
+  h->exit_ticket = h->canvas_ticket + cfg->B;
+  h->status = reinterpret_cast<uint32_t*>(base + o_status);
+  h->prev_amax = reinterpret_cast<int32_t*>(base + o_prev);
+  h->stable = reinterpret_cast<int32_t*>(base + o_stable);
+  h->sample = reinterpret_cast<int32_t*>(base + o_sample);
+  h->pmax = reinterpret_cast<float*>(base + o_pmax);
+  h->stop_next = reinterpret_cast<uint8_t*>(base + o_stopn);
+  *out = h;
+  return EB_OK;
+}
+
+int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
+                           uint8_t* stop_flags, void* stream) {
+  if (!h || !canvas || !committed || !stop_flags) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  const eb_config_t& c = h->cfg;
+  ebk::init_canvas_kernel<<<c.B, 256, 0, (cudaStream_t)stream>>>(
+      canvas, committed, stop_flags, h->stable, h->stop_next, c.L, c.V, c.canvas_offset,
+      (uint32_t)(c.seed & 0xffffffffu), (uint32_t)(c.seed >> 32));
+  if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
+  h->last_step = -1;
+  return EB_OK;
+}
+
+int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, int32_t* canvas,
+                    uint8_t* committed, float* entropies, int32_t* argmax, uint8_t* stop_flags,
+                    void* stream) {
+  if (!h || !logits || !canvas || !committed || !entropies || !argmax || !stop_flags)
+    return EB_ERR_INVALID_ARG;
+  if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
+  const eb_config_t& c = h->cfg;
+  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
+  if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  if (step == 0) {  // tickets are self-resetting; clear them anyway at a restart
+    if (cudaMemsetAsync(h->row_ticket, 0, h->tickets_bytes, st) != cudaSuccess) return EB_ERR_CUDA;
+  }
+
+  const double T = c.greedy ? 1.0
+                   : c.num_steps <= 1
+                       ? c.t_max
+                       : c.t_max + (c.t_min - c.t_max) * (double)step / (double)(c.num_steps - 1);
+  StepArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.logits = logits;
+  a.canvas = canvas;
+  a.committed = committed;
+  a.H_out = entropies;
+  a.amax_out = argmax;
+  a.stop_flags = stop_flags;
+  a.partials = h->partials;
+  a.row_ticket = h->row_ticket;
+  a.canvas_ticket = h->canvas_ticket;
+  a.exit_ticket = h->exit_ticket;
+  a.prev_amax = h->prev_amax;
+  a.stable = h->stable;
+  a.sample = h->sample;
+  a.pmax = h->pmax;
+  a.stop_next = h->stop_next;
+  a.status = h->status;
+  a.B = c.B;
+  a.L = c.L;
+  a.V = c.V;
+  a.ng = h->ng;
+  a.s = step;
+  a.N = c.num_steps;
+  a.max_segs = h->max_segs;
+  a.rule = c.rule;
+  a.quota = c.quota;
+  a.stability_steps = c.stability_steps;
+  a.greedy = c.greedy;
+  a.stop_enabled = c.stop_entropy >= 0.0 ? 1 : 0;
+  a.canvas_offset = c.canvas_offset;
+  a.c2d = 1.4426950408889634 / T;
+  a.c2 = (float)a.c2d;
+  a.iT = (float)(1.0 / T);
+  a.gamma = c.entropy_bound;
+  a.tau = c.stop_entropy;
+  a.theta = c.threshold;
+  a.key0 = (uint32_t)(c.seed & 0xffffffffu);
+  a.key1 = (uint32_t)(c.seed >> 32);
+
+  const size_t elt = dtype == EB_F32 ? 4 : 2;
+  const bool tma = ((uintptr_t)logits % 16 == 0) && (((size_t)c.V * elt) % 16 == 0);
+  const KernelCfg& kc = h->k[dtype][tma ? 1 : 0];
+  void* args[] = {&a};
+  if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::kThreads), args, kc.smem, st) !=
+      cudaSuccess)
+    return EB_ERR_CUDA;
+  h->last_step = step;
+  return EB_OK;
+}
+
+int eb_canvas_done(eb_sampler_t* h, const uint8_t* stop_flags, int b, int* done, void* stream) {
+  if (!h || !stop_flags || !done) return EB_ERR_INVALID_ARG;
+  if (b < -1 || b >= h->cfg.B) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const int n = h->cfg.B;
+  uint8_t local[64];
+  uint8_t* host = n <= 64 ? local : new (std::nothrow) uint8_t[n];
+  if (!host) return EB_ERR_OUT_OF_MEMORY;
+  uint32_t status = 0;
+  int rc = EB_OK;
+  if (cudaMemcpyAsync(host, stop_flags, (size_t)n, cudaMemcpyDeviceToHost, st) != cudaSuccess ||
+      cudaMemcpyAsync(&status, h->status, sizeof(status), cudaMemcpyDeviceToHost, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    rc = EB_ERR_CUDA;
+  } else {
+    int d = 1;
+    if (b >= 0) {
+      d = host[b] != 0;
+    } else {
+      for (int i = 0; i < n; ++i) d &= host[i] != 0;
+    }
+    *done = d;
+    if (status != 0) rc = EB_ERR_DEVICE_STATUS;
+  }
+  if (host != local) delete[] host;
+  return rc;
+}
+
+int eb_sampler_status(eb_sampler_t* h, uint32_t* status, int clear, void* stream) {
+  if (!h || !status) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  if (cudaMemcpyAsync(status, h->status, sizeof(uint32_t), cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return EB_ERR_CUDA;
+  if (clear && cudaMemsetAsync(h->status, 0, sizeof(uint32_t), st) != cudaSuccess)
+    return EB_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return EB_ERR_CUDA;
+  return EB_OK;
+}
+
+int eb_sampler_draws(eb_sampler_t* h, int32_t* sample, float* pmax, void* stream) {
+  if (!h) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BL = (size_t)h->cfg.B * (size_t)h->cfg.L;
+  if (sample &&
+      cudaMemcpyAsync(sample, h->sample, BL * sizeof(int32_t), cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+    return EB_ERR_CUDA;
+  if (pmax &&
+      cudaMemcpyAsync(pmax, h->pmax, BL * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
+          cudaSuccess)
+    return EB_ERR_CUDA;
+  return EB_OK;
+}
+
+int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int32_t* stable,
+                         int next_step, void* stream) {
+  if (!h || !prev_argmax) return EB_ERR_INVALID_ARG;
+  if (next_step < 0 || next_step >= h->cfg.num_steps) return EB_ERR_INVALID_ARG;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+  const size_t BL = (size_t)h->cfg.B * (size_t)h->cfg.L;
+  if (cudaMemcpyAsync(h->prev_amax, prev_argmax, BL * sizeof(int32_t), cudaMemcpyDeviceToDevice,
+                      st) != cudaSuccess)
+    return EB_ERR_CUDA;
+  if (stable) {
+    if (cudaMemcpyAsync(h->stable, stable, (size_t)h->cfg.B * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return EB_ERR_CUDA;
+  } else if (cudaMemsetAsync(h->stable, 0, (size_t)h->cfg.B * sizeof(int32_t), st) !=
+             cudaSuccess) {
+    return EB_ERR_CUDA;
+  }
+  if (cudaMemsetAsync(h->row_ticket, 0, h->tickets_bytes, st) != cudaSuccess) return EB_ERR_CUDA;
+  h->last_step = next_step - 1;
+  return EB_OK;
+}
+
+size_t eb_sampler_workspace_bytes(const eb_sampler_t* h) { return h ? h->ws_bytes : 0; }
+
+void eb_sampler_destroy(eb_sampler_t* h) {
+  if (!h) return;
+  {
+    DeviceGuard guard(h->device);
+    if (h->ws) cudaFree(h->ws);
+  }
+  delete h;
+}
+
+const char* eb_strerror(int code) {
+  switch (code) {
+    case EB_OK: return "ok";
+    case EB_ERR_INVALID_ARG: return "invalid argument";
+    case EB_ERR_CUDA: return "CUDA runtime error";
+    case EB_ERR_OUT_OF_MEMORY: return "out of device memory";
+    case EB_ERR_STEP_ORDER: return "step is neither 0 nor the previous step + 1";
+    case EB_ERR_UNSUPPORTED: return "unsupported dtype or device";
+    case EB_ERR_OVERFLOW: return "sizes exceed the library limits";
+    case EB_ERR_DEVICE_STATUS: return "a kernel reported a problem (status word non-zero)";
+    default: return "unknown status";
+  }
+}
+
+int eb_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,191 @@
+/*
+ * eb_sampler.h -- C ABI of the B200 entropy-bound (EB) canvas sampler.
+ *
+ * One call of eb_sampler_step performs one denoising step of DiffusionGemma's
+ * multi-canvas sampler on decoder logits [B canvases, L positions, V vocab]:
+ * tempered softmax entropy and argmax of every position, a categorical draw
+ * for every open position, the commit rule, the adaptive stop and the
+ * renoise of every position left open.
+ *
+ * Where the operation is defined (pages cited by title and section):
+ *   DiffusionGemma model card (Hugging Face / ai.google.dev), "Best
+ *   practices, 1. Diffusion sampling settings": at most 48 denoising steps,
+ *   temperature falling linearly 0.8 -> 0.4 for logit shaping, each step
+ *   selects the lowest-entropy tokens while the bound stays at
+ *   entropy_bound = 0.1, unselected tokens are fully renoised, and sampling
+ *   stops early once the canvas mean entropy is below 0.005 and the top
+ *   prediction is unchanged over two consecutive steps.
+ *   Same card, model summary table: canvas length 256, vocabulary ~262K.
+ *   diffusers v0.43.0 "DiffusionGemma" pipeline page, "Schedulers":
+ *   EntropyBoundScheduler (joint entropy of the committed positions under
+ *   entropy_bound; t_max 0.8 at the first step to t_min 0.4 at the last),
+ *   BlockRefinementScheduler (commit above `threshold` plus a uniform
+ *   per-step quota; greedy at temperature 0.0); "Adaptive stopping"
+ *   (stability_threshold, confidence_threshold on the scheduler-shaped
+ *   logits, per-sample freeze); "Static cache and compilation" (fixed shapes,
+ *   graph capture, the logits buffer is reused and must not be modified);
+ *   "Callbacks" (the canvas lives in caller tensors between steps).
+ *
+ * Conventions shared by every entry point:
+ *   - Every tensor argument is a DEVICE pointer owned by the caller (e.g. a
+ *     torch tensor's data_ptr()), row-major and contiguous:
+ *       logits     [B][L][V]  fp32 or bf16, read-only, 16-byte aligned for the
+ *                  bulk-copy path (other alignments use a slower load path)
+ *       canvas     [B][L] int32 tokens in [0, V), in/out
+ *       committed  [B][L] uint8 0/1, in/out, never reverts within a canvas
+ *       entropies  [B][L] fp32 out, nats, of softmax(logits / T_step)
+ *       argmax     [B][L] int32 out, lowest id among equal maxima
+ *       stop_flags [B] uint8 in/out: 0 active, else an EB_STOP_* reason
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy stream).
+ *   - Every function returns an int status (EB_OK = 0); nothing throws.
+ *   - A handle owns its device workspace; one handle per stream at a time;
+ *     handles are not thread-safe.
+ *   - Canvas b of a handle is canvas (canvas_offset + b) of the whole job;
+ *     all random draws are keyed by that global index, so a batch split
+ *     across devices gives the same bits as one device.
+ */
+#ifndef EB_SAMPLER_H
+#define EB_SAMPLER_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct eb_sampler eb_sampler_t;
+
+typedef enum { EB_F32 = 0, EB_BF16 = 1 } eb_dtype_t;
+
+/* Commit rules.  ENTROPY_BOUND: sort open positions by (entropy, position)
+   and commit the longest prefix whose entropy sum stays <= entropy_bound,
+   at least one position.  ENTROPY_BOUND_MI: the prefix's entropy sum minus
+   its largest entropy stays <= entropy_bound (the model cards' "mutual
+   information bound" wording).  BLOCK_REFINEMENT: open positions with
+   max probability >= threshold plus the next `quota` by (-pmax, position). */
+typedef enum {
+  EB_RULE_ENTROPY_BOUND = 0,
+  EB_RULE_BLOCK_REFINEMENT = 1,
+  EB_RULE_ENTROPY_BOUND_MI = 2
+} eb_rule_t;
+
+enum {
+  EB_OK = 0,
+  EB_ERR_INVALID_ARG = 1,    /* null pointer, bad size, bad config value */
+  EB_ERR_CUDA = 2,           /* a CUDA runtime call failed */
+  EB_ERR_OUT_OF_MEMORY = 3,  /* workspace allocation failed */
+  EB_ERR_STEP_ORDER = 4,     /* step is neither 0 nor previous step + 1 */
+  EB_ERR_UNSUPPORTED = 5,    /* unsupported dtype or device */
+  EB_ERR_OVERFLOW = 6,       /* sizes exceed the documented limits */
+  EB_ERR_DEVICE_STATUS = 7   /* a kernel reported a problem (see eb_sampler_status) */
+};
+
+/* Bits of the device status word. */
+enum {
+  EB_STATUS_BAD_TOKEN = 1,   /* a committed position held a token outside [0, V) */
+  EB_STATUS_NONFINITE = 2,   /* a row produced a non-finite softmax sum */
+  EB_STATUS_TIMEOUT = 4      /* an internal bounded wait gave up */
+};
+
+/* Stop reasons written to stop_flags. */
+enum {
+  EB_STOP_ACTIVE = 0,
+  EB_STOP_ADAPTIVE = 1,      /* adaptive stop fired; open positions took the argmax */
+  EB_STOP_ALL_COMMITTED = 2, /* the commit rule left nothing open */
+  EB_STOP_LAST_STEP = 3      /* step num_steps-1 committed every open position */
+};
+
+/* Size of the vocabulary groups of the two-level Gumbel-max draw. */
+#define EB_GUMBEL_GROUP 64
+
+/* Limits checked by eb_sampler_init. */
+#define EB_MAX_CANVASES 4096
+#define EB_MAX_POSITIONS 1024
+
+typedef struct {
+  int32_t B;               /* canvases in this handle, 1..EB_MAX_CANVASES */
+  int32_t L;               /* positions per canvas (256 on the model card), 1..EB_MAX_POSITIONS */
+  int32_t V;               /* vocabulary size (262144), >= 1 */
+  int32_t num_steps;       /* N, at most 48 on the model card, >= 1 */
+  double t_max, t_min;     /* temperature at step 0 and at step N-1 (0.8, 0.4), > 0 */
+  double entropy_bound;    /* gamma (0.1), >= 0 */
+  double stop_entropy;     /* tau (0.005); < 0 disables the adaptive stop */
+  int32_t stability_steps; /* consecutive unchanged-argmax steps required (1), >= 0 */
+  int32_t rule;            /* eb_rule_t */
+  double threshold;        /* block refinement confidence threshold (0.9) */
+  int32_t quota;           /* block refinement per-step quota (ceil(L/N) = 6), >= 0 */
+  int32_t greedy;          /* 1: temperature 0.0 -- shape with T = 1, commit argmax, no draw */
+  int32_t canvas_offset;   /* global index of canvas 0; offset + B <= 2^24 */
+  uint64_t seed;           /* key of every Philox4x32-10 draw */
+} eb_config_t;
+
+/* Fill *cfg with the model card's settings for B canvases of L x V. */
+void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V);
+
+/* Create a sampler on CUDA device `device` (the device must be sm_100).
+   Validates cfg, allocates and zeroes the workspace (partials, tickets,
+   previous argmax, stability counters, per-position draws, status word).
+   On success *out owns the handle (release with eb_sampler_destroy).
+   Errors: INVALID_ARG, OVERFLOW, UNSUPPORTED, OUT_OF_MEMORY, CUDA. */
+int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device);
+
+/* Start new canvases: canvas <- uniform-random tokens (generation starts from
+   a canvas of random placeholder tokens; uniform corruption, no mask token),
+   committed <- 0, stop_flags <- 0, and reset the stability state.  Enqueued
+   on `stream`, no host synchronisation. */
+int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
+                           uint8_t* stop_flags, void* stream);
+
+/* One denoising step `step` (0 .. num_steps-1) on `stream`.  `step` must be
+   0 (which restarts the step sequence) or the previous step + 1, else
+   EB_ERR_STEP_ORDER.  Canvases whose stop flag is set are skipped: their
+   logits are not read and their buffers are left untouched.  For every
+   other canvas: entropies/argmax of all L positions are written, open
+   positions are committed by the rule or renoised, and stop_flags[b] is set
+   when the canvas finishes.  Never synchronises the host, allocates nothing,
+   so a sequence of steps can be captured in a CUDA graph.  Kernel-side
+   problems set the status word instead of faulting (see eb_sampler_status).
+   Errors: INVALID_ARG, STEP_ORDER, UNSUPPORTED (dtype), CUDA (launch). */
+int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step,
+                    int32_t* canvas, uint8_t* committed, float* entropies,
+                    int32_t* argmax, uint8_t* stop_flags, void* stream);
+
+/* Synchronise `stream`, then report whether canvas b (or, for b = -1, every
+   canvas) has stopped, reading the device stop flags.  The only call that
+   waits for the device.  Returns EB_ERR_DEVICE_STATUS if the status word is
+   non-zero (the flags are still reported). */
+int eb_canvas_done(eb_sampler_t* h, const uint8_t* stop_flags, int b, int* done, void* stream);
+
+/* Synchronise `stream` and read the device status word (EB_STATUS_* bits);
+   clear it when `clear` is non-zero. */
+int eb_sampler_status(eb_sampler_t* h, uint32_t* status, int clear, void* stream);
+
+/* Copy the last step's per-position categorical draws ([B][L] int32, -1 for
+   positions that were committed before the step) and max probabilities
+   ([B][L] fp32) into caller device buffers on `stream`.  Either may be NULL. */
+int eb_sampler_draws(eb_sampler_t* h, int32_t* sample, float* pmax, void* stream);
+
+/* Resume support: overwrite the previous-step argmax ([B][L] int32, device)
+   and the per-canvas stability counters ([B] int32, device; NULL = zeros)
+   so that a trajectory checkpointed in caller buffers can continue at any
+   step.  Enqueued on `stream`. */
+int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int32_t* stable,
+                         int next_step, void* stream);
+
+/* Bytes of device workspace the handle holds. */
+size_t eb_sampler_workspace_bytes(const eb_sampler_t* h);
+
+/* Release the workspace and the handle (NULL is allowed). */
+void eb_sampler_destroy(eb_sampler_t* h);
+
+/* Static description of a status code. */
+const char* eb_strerror(int code);
+
+/* ABI version (major * 100 + minor). */
+int eb_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,381 @@
+"""GPU parity: the CUDA sampler (through the C ABI) against the CPU oracle.
+
+Full element-by-element comparison over whole trajectories for configurations
+the oracle finishes in seconds (several tiles per row and a ragged last
+group), and sampled comparison at the full workload sizes the benchmark uses.
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle as O
+import synth
+from parity import (Stats, compare_canvas, compare_rows, h_tol, oracle_config)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def E():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA GPU")
+    from entropy_bound_canvas_b200 import build as B
+    B.build()
+    import entropy_bound_canvas_b200 as E
+    return E
+
+
+DEV = "cuda:0"
+
+
+def tdtype(w):
+    return torch.float32 if w.dtype == synth.F32 else torch.bfloat16
+
+
+def host_logits(t):
+    """Device logits -> numpy (float32, or uint16 bf16 bits)."""
+    if t.dtype == torch.bfloat16:
+        return t.view(torch.int16).cpu().numpy().view(np.uint16)
+    return t.cpu().numpy()
+
+
+def alloc_logits(w, nb=None, byte_offset=0):
+    nb = w.B if nb is None else nb
+    n = nb * w.L * w.V
+    if byte_offset == 0:
+        return torch.empty((nb, w.L, w.V), dtype=tdtype(w), device=DEV)
+    raw = torch.empty(n * w.elt + 64, dtype=torch.uint8, device=DEV)
+    return raw[byte_offset:byte_offset + n * w.elt].view(tdtype(w)).view(nb, w.L, w.V)
+
+
+def make_sampler(E, w, **over):
+    cfg = w.sampler_config()
+    cfg.update(over)
+    return E.EBSampler(w.B, w.L, w.V, device=DEV, **cfg)
+
+
+def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=3):
+    """Whole trajectory, every canvas, every position compared with the oracle."""
+    eb = make_sampler(E, w, canvas_offset=canvas_offset)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    st = O.State(oracle_config(w, canvas_offset=canvas_offset)).init()
+    torch.cuda.synchronize()
+    assert np.array_equal(canvas.cpu().numpy(), st.canvas)
+    assert not committed.cpu().numpy().any() and not stop.cpu().numpy().any()
+    logits = alloc_logits(w, byte_offset=byte_offset)
+    f32 = w.dtype == synth.F32
+    stats = Stats()
+    prev_H = None
+    for s in range(w.num_steps):
+        synth.generate_device(w, s, logits, b0=canvas_offset)
+        eb.step(logits, s, canvas, committed, H, amax, stop)
+        smp, pm = eb.draws()
+        torch.cuda.synchronize()
+        lg = host_logits(logits)
+        Hg, amg, cvg, cmg, spg = (H.cpu().numpy(), amax.cpu().numpy(), canvas.cpu().numpy(),
+                                  committed.cpu().numpy(), stop.cpu().numpy())
+        smg, pmg = smp.cpu().numpy(), pm.cpu().numpy()
+        for i in range(w.B):
+            if st.stop[i]:
+                assert spg[i] == st.stop[i]
+                assert np.array_equal(cvg[i], st.canvas[i]) and cmg[i].all()
+                assert np.array_equal(Hg[i], prev_H[i])  # untouched once stopped
+                continue
+            out = O.step_canvas(st, i, lg[i], s)
+            compare_rows(stats, i, s, Hg[i], amg[i], pmg[i], smg[i], out, range(w.L), f32,
+                         out["open_before"])
+            differ = bool(np.any((smg[i] != out["sample"]) & out["open_before"]))
+            compare_canvas(stats, st, i, s, (cvg[i], cmg[i], spg[i]), out["margins"], differ)
+            if st.stop[i]:
+                stats.stop_steps[i] = s
+        prev_H = Hg.copy()
+        if st.stop.all():
+            assert eb.done(stop)
+            break
+    assert st.stop.all(), "every canvas stops by the last step"
+    assert stats.resyncs <= max_resyncs, stats
+    eb.close()
+    return stats
+
+
+# ----------------------------------------------------------------------------- full parity
+
+MID = synth.WORKLOADS["canvas"].replace(name="mid", B=3, L=64, V=8232, num_steps=24)
+
+
+@pytest.mark.parametrize("name,w", [
+    ("tiny", synth.WORKLOADS["tiny"]),
+    ("mid_bf16_eb", MID),
+    ("mid_f32_eb", MID.replace(dtype=synth.F32, seed=7)),
+    ("mid_bf16_mi", MID.replace(rule=O.RULE_EB_MI, seed=8)),
+    ("mid_bf16_br_greedy", MID.replace(rule=O.RULE_BR, greedy=1, quota=3, seed=9)),
+    ("mid_f32_br_sampled", MID.replace(dtype=synth.F32, rule=O.RULE_BR, quota=2, seed=10,
+                                       t_max=1.0, t_min=1.0)),
+    ("mid_zipf_f32", MID.replace(kind=synth.ZIPF, dtype=synth.F32, seed=11, B=2)),
+    ("mid_stop_disabled", MID.replace(stop_entropy=-1.0, seed=12, B=2, num_steps=10)),
+    ("mid_small_V", MID.replace(V=40, L=100, B=2, seed=13)),
+])
+def test_full_parity(E, name, w):
+    stats = run_full(E, w)
+    print(name, stats)
+
+
+def test_full_parity_unaligned_rows(E):
+    """Odd V (rows not 16-byte aligned): the element-load path."""
+    stats = run_full(E, MID.replace(V=5001, B=2, seed=14))
+    print(stats)
+
+
+def test_full_parity_offset_base_pointer(E):
+    """Logits base 2 bytes off a 16-byte boundary: the element-load path."""
+    stats = run_full(E, MID.replace(B=2, seed=15), byte_offset=2)
+    print(stats)
+
+
+def test_full_parity_canvas_offset(E):
+    stats = run_full(E, MID.replace(B=2, seed=16), canvas_offset=5)
+    print(stats)
+
+
+# ----------------------------------------------------------------------------- full size, sampled
+
+def run_sampled(E, w, canvases, n_rows=4, n_new=8, steps=None, rng_seed=0):
+    """Full-size trajectory; per step the oracle checks a few positions of the
+    tracked canvases one by one and re-derives every canvas decision from the
+    GPU's per-position outputs."""
+    rng = np.random.default_rng(rng_seed)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    st = O.State(oracle_config(w), canvases=canvases).init()
+    torch.cuda.synchronize()
+    assert np.array_equal(canvas.cpu().numpy()[canvases], st.canvas)
+    logits = alloc_logits(w)
+    f32 = w.dtype == synth.F32
+    stats = Stats()
+    N = w.num_steps if steps is None else steps
+    for s in range(N):
+        synth.generate_device(w, s, logits)
+        cm_before = committed.cpu().numpy()
+        eb.step(logits, s, canvas, committed, H, amax, stop)
+        smp, pm = eb.draws()
+        torch.cuda.synchronize()
+        Hg, amg, cvg, cmg, spg = (H.cpu().numpy(), amax.cpu().numpy(), canvas.cpu().numpy(),
+                                  committed.cpu().numpy(), stop.cpu().numpy())
+        smg, pmg = smp.cpu().numpy(), pm.cpu().numpy()
+        T = O.temperature(st.cfg, s)
+        for i, b in enumerate(canvases):
+            if st.stop[i]:
+                assert spg[b] == st.stop[i]
+                continue
+            new = np.nonzero(cmg[b] & ~cm_before[b])[0]
+            rows = set(rng.choice(w.L, n_rows, replace=False).tolist())
+            rows |= set(rng.permutation(new)[:n_new].tolist())
+            out = {k: np.zeros(w.L) for k in ("H", "pmax", "sample_margin")}
+            out.update(amax=np.zeros(w.L, np.int64), sample=np.full(w.L, -1, np.int64),
+                       sample_group=np.zeros(w.L, np.int64))
+            open_before = cm_before[b] == 0
+            for l in sorted(rows):
+                row = host_logits(logits[b, l])
+                Hh, pmh, amh, _ = O.row_stats(row, 1.0 / T)
+                out["H"][l], out["pmax"][l], out["amax"][l] = Hh, pmh, amh
+                if open_before[l]:
+                    if w.greedy:
+                        out["sample"][l], out["sample_margin"][l] = amh, np.inf
+                    else:
+                        x, mgn, grp = O.sample(st.cfg, row, 1.0 / T, b, l, s)
+                        out["sample"][l], out["sample_margin"][l], out["sample_group"][l] = x, mgn, grp
+            compare_rows(stats, b, s, Hg[b], amg[b], pmg[b], smg[b], out, sorted(rows), f32,
+                         open_before)
+            mg = O.canvas_decide(st, i, s, Hg[b].astype(np.float64), amg[b],
+                                 pmg[b].astype(np.float64), smg[b])
+            compare_canvas(stats, st, i, s, (cvg[b], cmg[b], spg[b]), mg, False)
+            if st.stop[i]:
+                stats.stop_steps[b] = s
+        if spg.all():
+            assert eb.done(stop)
+            break
+    eb.close()
+    return stats, stop.cpu().numpy()
+
+
+@pytest.mark.parametrize("name,canvases,steps", [
+    ("canvas", [0], None),
+    ("serve", [0, 3, 7], None),
+    ("br", [0, 3], None),
+    ("stress", [0, 31], 12),
+])
+def test_full_size_sampled(E, name, canvases, steps):
+    w = synth.WORKLOADS[name]
+    stats, stop = run_sampled(E, w, canvases, steps=steps)
+    print(name, stats)
+    assert stats.resyncs <= 2, stats
+
+
+# ----------------------------------------------------------------------------- edge cases
+
+def test_init_canvas_matches_oracle(E):
+    w = MID.replace(B=5)
+    eb = make_sampler(E, w, canvas_offset=11)
+    canvas, committed, stop = eb.new_canvas()
+    st = O.State(oracle_config(w, canvas_offset=11)).init()
+    torch.cuda.synchronize()
+    assert np.array_equal(canvas.cpu().numpy(), st.canvas)
+    assert (canvas.cpu().numpy() < w.V).all()
+
+
+def test_step_order_and_arguments(E):
+    w = MID.replace(B=1)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    logits = alloc_logits(w)
+    synth.generate_device(w, 0, logits)
+    with pytest.raises(E.EBError) as ei:
+        eb.step(logits, 3, canvas, committed, H, amax, stop)
+    assert ei.value.code == 4
+    with pytest.raises(E.EBError) as ei:
+        eb.step(logits, w.num_steps, canvas, committed, H, amax, stop)
+    assert ei.value.code == 1
+    assert eb.step_ptr(0, 1, 0, canvas.data_ptr(), committed.data_ptr(), H.data_ptr(),
+                       amax.data_ptr(), stop.data_ptr()) == 1
+    assert eb.step_ptr(logits.data_ptr(), 7, 0, canvas.data_ptr(), committed.data_ptr(),
+                       H.data_ptr(), amax.data_ptr(), stop.data_ptr()) == 5
+    eb.step(logits, 0, canvas, committed, H, amax, stop)
+    eb.step(logits, 1, canvas, committed, H, amax, stop)
+    with pytest.raises(E.EBError):
+        eb.step(logits, 1, canvas, committed, H, amax, stop)
+    eb.step(logits, 0, canvas, committed, H, amax, stop)  # restart is allowed
+    assert eb.status() == 0
+
+
+def test_bad_config_rejected(E):
+    with pytest.raises(E.EBError):
+        E.EBSampler(1, 0, 100, device=DEV)
+    with pytest.raises(E.EBError):
+        E.EBSampler(1, 2000, 100, device=DEV)
+    with pytest.raises(E.EBError):
+        E.EBSampler(1, 16, 100, device=DEV, t_max=-1.0)
+
+
+def test_stopped_canvas_is_skipped(E):
+    w = MID.replace(B=3, seed=21)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    H.fill_(-7.0)
+    amax.fill_(-9)
+    stop[1] = 2
+    before = (canvas[1].clone(), committed[1].clone())
+    logits = alloc_logits(w)
+    for s in range(4):
+        synth.generate_device(w, s, logits)
+        eb.step(logits, s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    assert torch.equal(canvas[1], before[0]) and torch.equal(committed[1], before[1])
+    assert (H[1] == -7.0).all() and (amax[1] == -9).all() and int(stop[1]) == 2
+    assert (H[0] >= 0).all() and (H[2] >= 0).all()
+
+
+def test_bad_committed_token_sets_status(E):
+    w = MID.replace(B=1, seed=22)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    committed[0, 3] = 1
+    canvas[0, 3] = w.V + 5
+    logits = alloc_logits(w)
+    synth.generate_device(w, 0, logits)
+    eb.step(logits, 0, canvas, committed, H, amax, stop)
+    assert eb.status(clear=True) & E.STATUS_BAD_TOKEN
+    assert eb.status() == 0
+    assert int(canvas[0, 3]) == w.V + 5  # committed tokens are never rewritten
+
+
+def test_stop_fires_on_predicted_step(E):
+    L, V = 16, 512
+    eb = E.EBSampler(1, L, V, device=DEV, num_steps=30, seed=5, entropy_bound=0.0)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    tgt = torch.arange(L, device=DEV) * 31 % V
+    fired = None
+    for s in range(30):
+        z = torch.zeros((1, L, V), dtype=torch.float32, device=DEV)
+        t = tgt if s >= 6 else (tgt + s) % V
+        z[0, torch.arange(L, device=DEV), t] = 40.0 if s >= 6 else 0.5
+        eb.step(z, s, canvas, committed, H, amax, stop)
+        if int(stop[0]):
+            fired = (s, int(stop[0]))
+            break
+    assert fired == (7, E.STOP_ADAPTIVE)
+    assert bool(committed.all())
+
+
+def test_sharded_canvases_equal_one_handle(E):
+    """Canvases split over two handles with canvas offsets give the same bits."""
+    w = MID.replace(B=4, seed=23, num_steps=8)
+    logits = alloc_logits(w)
+    one = make_sampler(E, w)
+    c1, m1, s1 = one.new_canvas()
+    H1, a1 = one.outputs()
+    parts = []
+    for r in range(2):
+        off, cnt = E.shard_canvases(w.B, 2, r)
+        wp = w.replace(B=cnt)
+        e = make_sampler(E, wp, canvas_offset=off)
+        c, m, s = e.new_canvas()
+        h, a = e.outputs()
+        parts.append((e, off, cnt, c, m, s, h, a))
+    for st in range(w.num_steps):
+        synth.generate_device(w, st, logits)
+        one.step(logits, st, c1, m1, H1, a1, s1)
+        for e, off, cnt, c, m, s, h, a in parts:
+            e.step(logits[off:off + cnt].contiguous(), st, c, m, h, a, s)
+    torch.cuda.synchronize()
+    for e, off, cnt, c, m, s, h, a in parts:
+        assert torch.equal(c, c1[off:off + cnt]) and torch.equal(m, m1[off:off + cnt])
+        assert torch.equal(s, s1[off:off + cnt]) and torch.equal(a, a1[off:off + cnt])
+        assert torch.allclose(h, H1[off:off + cnt], atol=1e-6, rtol=0)
+
+
+def test_deterministic_and_graph_capture(E):
+    w = MID.replace(B=2, seed=24, num_steps=12)
+    logits = torch.empty((w.num_steps, w.B, w.L, w.V), dtype=tdtype(w), device=DEV)
+    for s in range(w.num_steps):
+        synth.generate_device(w, s, logits[s])
+
+    def eager():
+        eb = make_sampler(E, w)
+        c, m, st = eb.new_canvas()
+        h, a = eb.outputs()
+        for s in range(w.num_steps):
+            eb.step(logits[s], s, c, m, h, a, st)
+        torch.cuda.synchronize()
+        return c, m, st, h, a
+
+    r1, r2 = eager(), eager()
+    for x, y in zip(r1, r2):
+        assert torch.equal(x, y)
+
+    eb = make_sampler(E, w)
+    c, m, st = eb.new_canvas()
+    h, a = eb.outputs()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(side):
+        eb.init_canvas(c, m, st)
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=side):
+            eb.init_canvas(c, m, st)
+            for s in range(w.num_steps):
+                eb.step(logits[s], s, c, m, h, a, st)
+    for _ in range(2):
+        g.replay()
+        torch.cuda.synchronize()
+        for x, y in zip((c, m, st, h, a), r1):
+            assert torch.equal(x, y)
+    del g
