@@ -52,6 +52,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=48)
+    p.add_argument("--profile", action="store_true",
+                   help="small case for ncu: logits of steps 0-2 only, three eager steps")
     return p.parse_args()
 
 
@@ -161,10 +163,13 @@ def run_reference(args):
         rows_per_step = max(1, budget_rows // total)
     st = O.State(cfg).init()
     times = []
+    cache = {}
     for i in range(total):
         s = i % w.num_steps
-        l0 = (i * 37) % (w.L - rows_per_step + 1)
-        rows = synth.generate_host(w, s, 0, 1, l0, rows_per_step)[0]
+        l0 = (s * 37) % (w.L - rows_per_step + 1)
+        if (s, l0) not in cache:
+            cache[(s, l0)] = synth.generate_host(w, s, 0, 1, l0, rows_per_step)[0]
+        rows = cache[(s, l0)]
         t0 = time.perf_counter()
         T = O.temperature(cfg, s)
         H = np.zeros(w.L)
@@ -425,8 +430,33 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_profile_case():
+    """Three eager steps of the benchmark workload (about 0.4 GB on the device)."""
+    import torch
+
+    import entropy_bound_canvas_b200 as E
+    import synth
+    w = synth.WORKLOADS[WORKLOAD]
+    dev = torch.device("cuda", 0)
+    logits = [torch.empty((w.B, w.L, w.V), dtype=torch.bfloat16, device=dev) for _ in range(3)]
+    for s in range(3):
+        synth.generate_device(w, s, logits[s])
+    eb = E.EBSampler(w.B, w.L, w.V, device=dev, **w.sampler_config())
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    for s in range(3):
+        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    assert eb.status() == 0
+    eb.close()
+    print("profile case done")
+
+
 def main():
     args = parse()
+    if args.profile:
+        run_profile_case()
+        return
     if args.impl == "reference":
         run_reference(args)
     else:

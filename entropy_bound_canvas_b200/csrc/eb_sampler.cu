@@ -285,8 +285,7 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.greedy = c.greedy;
   a.stop_enabled = c.stop_entropy >= 0.0 ? 1 : 0;
   a.canvas_offset = c.canvas_offset;
-  a.c2d = 1.4426950408889634 / T;
-  a.c2 = (float)a.c2d;
+  a.c2 = (float)(1.4426950408889634 / T);
   a.iT = (float)(1.0 / T);
   a.gamma = c.entropy_bound;
   a.tau = c.stop_entropy;

@@ -42,7 +42,6 @@ constexpr int kThreads = kConsumers + 32;
 constexpr int kTileGroups = kConsumers;
 constexpr int kStages = 3;
 constexpr int kMaxL = 1024;
-constexpr int kPerThread = kMaxL / kConsumers;
 
 enum : uint32_t { kStatusBadToken = 1, kStatusNonFinite = 2, kStatusTimeout = 4 };
 enum : int { kF32 = 0, kBF16 = 1 };
@@ -51,14 +50,16 @@ enum : int { kRuleEB = 0, kRuleBR = 1, kRuleMI = 2 };
 __host__ __device__ constexpr int elt_bytes(int dt) { return dt == kF32 ? 4 : 2; }
 __host__ __device__ constexpr int tile_bytes(int dt) { return kTileGroups * kGroup * elt_bytes(dt); }
 
-// Per-(row, CTA segment) partial: S = sum 2^d, W = sum 2^d d with
-// d = (z - zmax) c2, plus argmax, the fp32 sums of the group that holds the
-// argmax (as they entered S and W), and the best Gumbel group.
+// Per-(row, CTA segment) partial, relative to the segment's maximum logit
+// zmax with d = (z - zmax) c2 (log2 units): the fp32 sums of the group that
+// holds the argmax (Stop = sum 2^d, Wtop = sum 2^d d) kept apart from the sums
+// of everything else (Srest, Wrest), so that the row combine can replace the
+// top group by an exact recomputation; plus the best Gumbel group.
 struct Partial {
-  double S, W;
   float zmax;
-  int amax;
+  int agrp;  // lowest group index holding zmax
   float Stop, Wtop;
+  float Srest, Wrest;
   float gscore;
   int gidx;
 };
@@ -84,7 +85,6 @@ struct StepArgs {
   int rule, quota, stability_steps, greedy, stop_enabled;
   int canvas_offset;
   float c2, iT;
-  double c2d;
   double gamma, tau, theta;
   uint32_t key0, key1;
 };
@@ -145,22 +145,43 @@ struct Tile {
   long long r;  // active row index
   int j0;       // first group of the tile within the row
   int cnt;      // groups in the tile
+  int ai;       // index of the row's canvas in the active list
+  int l;        // position of the row
 };
 
+// Walks a CTA's group range tile by tile; divides only once, at the start.
 struct TileIter {
   unsigned long long g, g_hi;
-  int ng;
+  int ng, L;
+  long long r;
+  int j0, ai, l;
+  __device__ __forceinline__ TileIter(unsigned long long lo, unsigned long long hi, int ng_, int L_)
+      : g(lo), g_hi(hi), ng(ng_), L(L_) {
+    r = (long long)(lo / (unsigned long long)ng_);
+    j0 = (int)(lo - (unsigned long long)r * (unsigned long long)ng_);
+    ai = (int)(r / L_);
+    l = (int)(r - (long long)ai * L_);
+  }
   __device__ __forceinline__ bool next(Tile& t) {
     if (g >= g_hi) return false;
-    const unsigned long long r = g / (unsigned long long)ng;
-    const int j0 = (int)(g - r * (unsigned long long)ng);
     int cnt = ng - j0;
     if (cnt > kTileGroups) cnt = kTileGroups;
     if ((unsigned long long)cnt > g_hi - g) cnt = (int)(g_hi - g);
-    t.r = (long long)r;
+    t.r = r;
     t.j0 = j0;
     t.cnt = cnt;
+    t.ai = ai;
+    t.l = l;
     g += (unsigned long long)cnt;
+    j0 += cnt;
+    if (j0 == ng) {
+      j0 = 0;
+      ++r;
+      if (++l == L) {
+        l = 0;
+        ++ai;
+      }
+    }
     return true;
   }
 };
@@ -170,15 +191,26 @@ struct TileIter {
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ Partial empty_partial() {
   Partial p;
-  p.S = 0.0;
-  p.W = 0.0;
   p.zmax = -INFINITY;
-  p.amax = 0x7fffffff;
+  p.agrp = 0x7fffffff;
   p.Stop = 0.f;
   p.Wtop = 0.f;
+  p.Srest = 0.f;
+  p.Wrest = 0.f;
   p.gscore = -INFINITY;
   p.gidx = 0x7fffffff;
   return p;
+}
+
+// Everything of `o` (top and rest), rescaled from o.zmax to zmax, added to
+// the rest sums of `a` (whose maximum zmax >= o.zmax).
+__device__ __forceinline__ void add_to_rest(Partial& a, const Partial& o, float c2) {
+  const float d = (o.zmax - a.zmax) * c2;
+  const float f = ex2(d);
+  const float S = o.Stop + o.Srest;
+  const float W = o.Wtop + o.Wrest;
+  a.Srest = fmaf(f, S, a.Srest);
+  a.Wrest = fmaf(f, fmaf(d, S, W), a.Wrest);
 }
 
 __device__ __forceinline__ void merge(Partial& a, const Partial& b, float c2) {
@@ -188,38 +220,33 @@ __device__ __forceinline__ void merge(Partial& a, const Partial& b, float c2) {
   }
   if (!(b.zmax > -INFINITY)) return;
   if (!(a.zmax > -INFINITY)) {
-    a.S = b.S;
-    a.W = b.W;
-    a.zmax = b.zmax;
-    a.amax = b.amax;
-    a.Stop = b.Stop;
-    a.Wtop = b.Wtop;
+    const float gs = a.gscore;
+    const int gi = a.gidx;
+    a = b;
+    a.gscore = gs;
+    a.gidx = gi;
     return;
   }
-  const bool b_top = b.zmax > a.zmax || (b.zmax == a.zmax && b.amax < a.amax);
-  const float M = fmaxf(a.zmax, b.zmax);
-  const float da = (a.zmax - M) * c2, db = (b.zmax - M) * c2;
-  const double fa = (double)ex2(da), fb = (double)ex2(db);
-  const double S = fa * a.S + fb * b.S;
-  const double W = fa * (a.W + (double)da * a.S) + fb * (b.W + (double)db * b.S);
-  a.S = S;
-  a.W = W;
+  const bool b_top = b.zmax > a.zmax || (b.zmax == a.zmax && b.agrp < a.agrp);
   if (b_top) {
-    a.zmax = b.zmax;
-    a.amax = b.amax;
-    a.Stop = b.Stop;
-    a.Wtop = b.Wtop;
+    Partial t = b;
+    t.gscore = a.gscore;
+    t.gidx = a.gidx;
+    add_to_rest(t, a, c2);
+    a = t;
+  } else {
+    add_to_rest(a, b, c2);
   }
 }
 
 __device__ __forceinline__ Partial shfl_partial(const Partial& p, int mask_lane) {
   Partial q;
-  q.S = __shfl_xor_sync(0xffffffffu, p.S, mask_lane);
-  q.W = __shfl_xor_sync(0xffffffffu, p.W, mask_lane);
   q.zmax = __shfl_xor_sync(0xffffffffu, p.zmax, mask_lane);
-  q.amax = __shfl_xor_sync(0xffffffffu, p.amax, mask_lane);
+  q.agrp = __shfl_xor_sync(0xffffffffu, p.agrp, mask_lane);
   q.Stop = __shfl_xor_sync(0xffffffffu, p.Stop, mask_lane);
   q.Wtop = __shfl_xor_sync(0xffffffffu, p.Wtop, mask_lane);
+  q.Srest = __shfl_xor_sync(0xffffffffu, p.Srest, mask_lane);
+  q.Wrest = __shfl_xor_sync(0xffffffffu, p.Wrest, mask_lane);
   q.gscore = __shfl_xor_sync(0xffffffffu, p.gscore, mask_lane);
   q.gidx = __shfl_xor_sync(0xffffffffu, p.gidx, mask_lane);
   return q;
@@ -242,7 +269,6 @@ struct GroupStat {
   float m;    // raw maximum
   float S;    // sum 2^d, d = (z - m) c2
   float W;    // sum 2^d d
-  int first;  // lowest index in the group holding m (only when m > cur_max)
 };
 
 // Lane-wise maximum of two packed bf16 pairs.
@@ -252,114 +278,120 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   return d;
 }
 
+// Packed fp32 pair arithmetic (sm_100): one instruction for two lanes.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "mov.b64 c, {%6, %7};\n\tfma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return r;
+}
+
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 r;
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(r.x), "=f"(r.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return r;
+}
+
+// Accumulates one pair of logits: d = z c2 - m c2, p = 2^d, S += p, W += p d.
+// The maximum itself gets d = the rounding residue of m c2 rather than 0;
+// the row combine recomputes the group holding the argmax exactly.
+__device__ __forceinline__ void acc_pair(float2 z, float2 c2v, float2 nmc, float2& S, float2& W) {
+  const float2 d = ffma2(z, c2v, nmc);
+  float2 p;
+  p.x = ex2(d.x);
+  p.y = ex2(d.y);
+  S = fadd2(S, p);
+  W = ffma2(p, d, W);
+}
+
 __device__ __forceinline__ float tree8(const float (&v)[8]) {
   return ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
 }
 
-// Full 64-element bf16 group in shared memory (128 bytes).  Pieces of 16
-// bytes are read in an order rotated by the thread index so that the eight
-// threads of a shared-memory phase hit eight different bank quads.
-__device__ __forceinline__ GroupStat group_bf16_full(const unsigned char* gp, int rot, float c2,
-                                                     float cur_max) {
+__device__ __forceinline__ float sum4(const float2 (&v)[4]) {
+  return ((v[0].x + v[0].y) + (v[1].x + v[1].y)) + ((v[2].x + v[2].y) + (v[3].x + v[3].y));
+}
+
+// Full 64-element bf16 group in shared memory (128 bytes), read twice (max,
+// then exponentials) to keep register use low.  Pieces of 16 bytes are read
+// in an order rotated by the thread index so that the eight threads of a
+// shared-memory phase hit eight different bank quads.
+__device__ __forceinline__ GroupStat group_bf16_full(const unsigned char* gp, int rot, float c2) {
   const uint4* q = reinterpret_cast<const uint4*>(gp);
-  uint32_t w[32];
+  uint32_t mx0, mx1;
+  {
+    const uint4 v = q[rot & 7];
+    mx0 = bf16x2_max(v.x, v.y);
+    mx1 = bf16x2_max(v.z, v.w);
+  }
+#pragma unroll
+  for (int k = 1; k < 8; ++k) {
+    const uint4 v = q[(k + rot) & 7];
+    mx0 = bf16x2_max(mx0, bf16x2_max(v.x, v.y));
+    mx1 = bf16x2_max(mx1, bf16x2_max(v.z, v.w));
+  }
+  const uint32_t mx = bf16x2_max(mx0, mx1);
+  const float m = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xffff0000u));
+  const float2 c2v = make_float2(c2, c2);
+  const float2 nmc = make_float2(-m * c2, -m * c2);
+
+  float2 S[4], W[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    S[i] = make_float2(0.f, 0.f);
+    W[i] = make_float2(0.f, 0.f);
+  }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     const uint4 v = q[(k + rot) & 7];
-    w[4 * k + 0] = v.x;
-    w[4 * k + 1] = v.y;
-    w[4 * k + 2] = v.z;
-    w[4 * k + 3] = v.w;
-  }
-  uint32_t mx = w[0];
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-  for (int i = 1; i < 32; ++i) mx = bf16x2_max(mx, w[i]);
-  const float m = fmaxf(__uint_as_float(mx << 16), __uint_as_float(mx & 0xffff0000u));
-
-  float s[8], ws[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s[i] = 0.f;
-    ws[i] = 0.f;
-  }
-#pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const float lo = __uint_as_float(w[i] << 16);
-    const float hi = __uint_as_float(w[i] & 0xffff0000u);
-    const float d0 = (lo - m) * c2;
-    const float d1 = (hi - m) * c2;
-    const float p0 = ex2(d0);
-    const float p1 = ex2(d1);
-    s[(2 * i) & 7] += p0;
-    ws[(2 * i) & 7] = fmaf(p0, d0, ws[(2 * i) & 7]);
-    s[(2 * i + 1) & 7] += p1;
-    ws[(2 * i + 1) & 7] = fmaf(p1, d1, ws[(2 * i + 1) & 7]);
+    for (int i = 0; i < 4; ++i) {
+      const float2 z = make_float2(__uint_as_float(w4[i] << 16), __uint_as_float(w4[i] & 0xffff0000u));
+      acc_pair(z, c2v, nmc, S[i], W[i]);
+    }
   }
   GroupStat g;
   g.m = m;
-  g.S = tree8(s);
-  g.W = tree8(ws);
-  g.first = kGroup;
-  if (m > cur_max) {
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const int base = ((k + rot) & 7) * 8;
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float lo = __uint_as_float(w[4 * k + i] << 16);
-        const float hi = __uint_as_float(w[4 * k + i] & 0xffff0000u);
-        const int e0 = base + 2 * i;
-        if (lo == m && e0 < g.first) g.first = e0;
-        if (hi == m && e0 + 1 < g.first) g.first = e0 + 1;
-      }
-    }
-  }
+  g.S = sum4(S);
+  g.W = sum4(W);
   return g;
 }
 
-// Full 64-element fp32 group in shared memory (256 bytes), read twice (max,
-// then exponentials) to keep register use low.
-__device__ __forceinline__ GroupStat group_f32_full(const unsigned char* gp, int rot, float c2,
-                                                    float cur_max) {
+// Full 64-element fp32 group in shared memory (256 bytes), read twice.
+__device__ __forceinline__ GroupStat group_f32_full(const unsigned char* gp, int rot, float c2) {
   const float4* q = reinterpret_cast<const float4*>(gp);
-  float m = -INFINITY;
+  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const float4 v = q[(k + rot) & 15];
-    m = fmaxf(m, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    m0 = fmaxf(m0, fmaxf(v.x, v.y));
+    m1 = fmaxf(m1, fmaxf(v.z, v.w));
   }
-  float s[8], ws[8];
+  const float m = fmaxf(m0, m1);
+  const float2 c2v = make_float2(c2, c2);
+  const float2 nmc = make_float2(-m * c2, -m * c2);
+  float2 S[4], W[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s[i] = 0.f;
-    ws[i] = 0.f;
+  for (int i = 0; i < 4; ++i) {
+    S[i] = make_float2(0.f, 0.f);
+    W[i] = make_float2(0.f, 0.f);
   }
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
     const float4 v = q[(k + rot) & 15];
-    const float z[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float d = (z[i] - m) * c2;
-      const float p = ex2(d);
-      s[(4 * k + i) & 7] += p;
-      ws[(4 * k + i) & 7] = fmaf(p, d, ws[(4 * k + i) & 7]);
-    }
+    acc_pair(make_float2(v.x, v.y), c2v, nmc, S[(2 * k) & 3], W[(2 * k) & 3]);
+    acc_pair(make_float2(v.z, v.w), c2v, nmc, S[(2 * k + 1) & 3], W[(2 * k + 1) & 3]);
   }
   GroupStat g;
   g.m = m;
-  g.S = tree8(s);
-  g.W = tree8(ws);
-  g.first = kGroup;
-  if (m > cur_max) {
-#pragma unroll 1
-    for (int e = 0; e < kGroup; ++e) {
-      if (reinterpret_cast<const float*>(gp)[e] == m) {
-        g.first = e;
-        break;
-      }
-    }
-  }
+  g.S = sum4(S);
+  g.W = sum4(W);
   return g;
 }
 
@@ -372,16 +404,9 @@ __device__ __forceinline__ float load_elem(const void* p, int e) {
 // Any group (partial last group of a row, or unaligned rows): element by
 // element through a generic pointer (shared or global memory).
 template <int DT>
-__device__ __noinline__ GroupStat group_scalar(const void* gp, int glen, float c2, float cur_max) {
+__device__ __noinline__ GroupStat group_scalar(const void* gp, int glen, float c2) {
   float m = -INFINITY;
-  int first = kGroup;
-  for (int e = 0; e < glen; ++e) {
-    const float z = load_elem<DT>(gp, e);
-    if (z > m) {
-      m = z;
-      first = e;
-    }
-  }
+  for (int e = 0; e < glen; ++e) m = fmaxf(m, load_elem<DT>(gp, e));
   float s[8], ws[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -398,32 +423,31 @@ __device__ __noinline__ GroupStat group_scalar(const void* gp, int glen, float c
   g.m = m;
   g.S = tree8(s);
   g.W = tree8(ws);
-  g.first = m > cur_max ? first : kGroup;
   return g;
 }
 
 // Fold one group into a thread's running partial (groups arrive in
 // increasing index order within a row segment, so a tie never moves the
 // argmax).
-__device__ __forceinline__ void fold_group(Partial& t, const GroupStat& g, int gbase, float c2) {
+__device__ __forceinline__ void fold_group(Partial& t, const GroupStat& g, int j, float c2) {
   if (g.m > t.zmax) {
     if (t.zmax > -INFINITY) {
       const float d = (t.zmax - g.m) * c2;
-      const double f = (double)ex2(d);
-      t.W = f * (t.W + (double)d * t.S);
-      t.S = f * t.S;
+      const float f = ex2(d);
+      const float S = t.Stop + t.Srest;
+      const float W = t.Wtop + t.Wrest;
+      t.Srest = f * S;
+      t.Wrest = f * fmaf(d, S, W);
     }
-    t.S += (double)g.S;
-    t.W += (double)g.W;
-    t.zmax = g.m;
-    t.amax = gbase + g.first;
     t.Stop = g.S;
     t.Wtop = g.W;
+    t.zmax = g.m;
+    t.agrp = j;
   } else {
     const float d = (g.m - t.zmax) * c2;
-    const double f = (double)ex2(d);
-    t.S += f * (double)g.S;
-    t.W += f * ((double)g.W + (double)d * (double)g.S);
+    const float f = ex2(d);
+    t.Srest = fmaf(f, g.S, t.Srest);
+    t.Wrest = fmaf(f, fmaf(d, g.S, g.W), t.Wrest);
   }
 }
 
@@ -501,41 +525,38 @@ __device__ __forceinline__ unsigned long long key_desc(float p, int l) {
 // ---------------------------------------------------------------------------
 // Canvas epilogue: stability, adaptive stop, commit rule, finalisation,
 // renoise.  Runs on the 128 consumer threads of the CTA that completed the
-// canvas's last row.
+// canvas's last row.  Kept compact (positions in rolled loops, values
+// re-read from L2) because it runs from a cold instruction cache.
 // ---------------------------------------------------------------------------
-__device__ void canvas_epilogue(const StepArgs& a, int bi, Ctrl* ctrl, unsigned long long* keys,
-                                unsigned long long* skeys, uint8_t* pick, int tid) {
+__device__ __noinline__ void canvas_epilogue(const StepArgs a, int bi, Ctrl* ctrl,
+                                             unsigned long long* keys, unsigned long long* skeys,
+                                             uint8_t* pick, int tid) {
   const int L = a.L;
   const size_t row0 = (size_t)bi * (size_t)L;
   const int lane = tid & 31, warp = tid >> 5;
+  const bool br = a.rule == kRuleBR;
 
-  float Hr[kPerThread];
-  int amr[kPerThread], smr[kPerThread];
-  float pmr[kPerThread];
-  bool openr[kPerThread];
+  // Pass 1: entropy sum, argmax stability, candidate counts.
   double sumH = 0.0;
   int neq = a.s < 1 ? 1 : 0;
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    const int l = tid + k * kConsumers;
-    openr[k] = false;
-    Hr[k] = 0.f;
-    amr[k] = 0;
-    smr[k] = 0;
-    pmr[k] = 0.f;
-    if (l < L) {
-      Hr[k] = __ldcg(a.H_out + row0 + l);
-      amr[k] = __ldcg(a.amax_out + row0 + l);
-      smr[k] = __ldcg(a.sample + row0 + l);
-      pmr[k] = __ldcg(a.pmax + row0 + l);
-      openr[k] = a.committed[row0 + l] == 0;
-      pick[l] = 0;
-      sumH += (double)Hr[k];
-      if (a.s >= 1 && amr[k] != a.prev_amax[row0 + l]) neq = 1;
-      if (!openr[k]) {
-        const int tok = a.canvas[row0 + l];
-        if (tok < 0 || tok >= a.V) atomicOr(a.status, kStatusBadToken);
-      }
+  int ncand = 0;
+#pragma unroll 1
+  for (int l = tid; l < L; l += kConsumers) {
+    const float H = __ldcg(a.H_out + row0 + l);
+    const int am = __ldcg(a.amax_out + row0 + l);
+    const bool open = a.committed[row0 + l] == 0;
+    pick[l] = 0;
+    sumH += (double)H;
+    if (a.s >= 1 && am != a.prev_amax[row0 + l]) neq = 1;
+    if (!open) {
+      const int tok = a.canvas[row0 + l];
+      if (tok < 0 || tok >= a.V) atomicOr(a.status, kStatusBadToken);
+    } else if (!br) {
+      ncand += (double)H <= a.gamma ? 1 : 0;
+    } else if ((double)__ldcg(a.pmax + row0 + l) >= a.theta) {
+      pick[l] = 1;
+    } else {
+      ++ncand;
     }
   }
   const double totH = block_sum(sumH, ctrl, tid);
@@ -544,43 +565,35 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, Ctrl* ctrl, unsigned 
   const double meanH = totH / (double)L;
   const bool fired = a.stop_enabled && stable_new >= a.stability_steps && meanH < a.tau;
   const bool last_step = a.s == a.N - 1;
-  const uint32_t bg = (uint32_t)(a.canvas_offset + bi);
-  int reason = 0;
 
-  if (fired) {
-#pragma unroll
-    for (int k = 0; k < kPerThread; ++k) {
-      const int l = tid + k * kConsumers;
-      if (l < L && openr[k]) {
-        a.canvas[row0 + l] = amr[k];
-        a.committed[row0 + l] = 1;
+  if (!fired) {
+    // Candidates: EB -- open positions with H <= gamma (no other can be in the
+    // prefix); BR -- open positions below the threshold (quota competitors).
+    int n_c = 0;
+    int pos = block_excl_scan(ncand, ctrl, tid, &n_c);
+#pragma unroll 1
+    for (int l = tid; l < L; l += kConsumers) {
+      if (a.committed[row0 + l] != 0) continue;
+      if (!br) {
+        const float H = __ldcg(a.H_out + row0 + l);
+        if ((double)H <= a.gamma) keys[pos++] = key_asc(H, l);
+      } else {
+        const float p = __ldcg(a.pmax + row0 + l);
+        if (!((double)p >= a.theta)) keys[pos++] = key_desc(p, l);
       }
     }
-    reason = 1;
-  } else {
-    if (a.rule == kRuleEB || a.rule == kRuleMI) {
-      // Candidates: open positions with H <= gamma (no other can be in the prefix).
-      int nmine = 0;
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        const int l = tid + k * kConsumers;
-        if (l < L && openr[k] && (double)Hr[k] <= a.gamma) ++nmine;
-      }
-      int n_c = 0;
-      int pos = block_excl_scan(nmine, ctrl, tid, &n_c);
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        const int l = tid + k * kConsumers;
-        if (l < L && openr[k] && (double)Hr[k] <= a.gamma) keys[pos++] = key_asc(Hr[k], l);
-      }
-      consumer_sync(kConsumers);
-      for (int c = tid; c < n_c; c += kConsumers) {
-        const unsigned long long kc = keys[c];
-        int rank = 0;
-        for (int j = 0; j < n_c; ++j) rank += keys[j] < kc;
-        skeys[rank] = kc;
-      }
-      consumer_sync(kConsumers);
+    consumer_sync(kConsumers);
+#pragma unroll 1
+    for (int c = tid; c < n_c; c += kConsumers) {
+      const unsigned long long kc = keys[c];
+      int rank = 0;
+#pragma unroll 4
+      for (int j = 0; j < n_c; ++j) rank += keys[j] < kc;
+      if (!br) skeys[rank] = kc;
+      else if (rank < a.quota) pick[(int)(kc & 0xffffffffu)] = 1;
+    }
+    consumer_sync(kConsumers);
+    if (!br) {
       // Longest prefix of the sorted candidates with cumulative H <= gamma.
       if (warp == 0) {
         const int chunk = (n_c + 31) / 32;
@@ -608,87 +621,54 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, Ctrl* ctrl, unsigned 
       consumer_sync(kConsumers);
       const int kpref = ctrl->kpref;
       for (int i = tid; i < kpref; i += kConsumers) pick[(int)(skeys[i] & 0xffffffffu)] = 1;
-      bool need_min = false;
-      bool only_noncand = false;
-      if (a.rule == kRuleEB) {
-        need_min = kpref == 0;
-      } else if (kpref < n_c) {
+      // EB with an empty prefix: the single lowest (H, l).  MI: the prefix
+      // plus the next position in (H, l) order.
+      const bool mi = a.rule == kRuleMI;
+      if (mi && kpref < n_c) {
         if (tid == 0) pick[(int)(skeys[kpref] & 0xffffffffu)] = 1;
-      } else {
-        need_min = true;
-        only_noncand = true;
-      }
-      if (need_min) {  // the lowest (H, l) among the open positions not yet chosen
+      } else if (kpref == 0 || mi) {
         unsigned long long best = ~0ull;
-#pragma unroll
-        for (int k = 0; k < kPerThread; ++k) {
-          const int l = tid + k * kConsumers;
-          if (l < L && openr[k] && (!only_noncand || !((double)Hr[k] <= a.gamma))) {
-            const unsigned long long kk = key_asc(Hr[k], l);
-            best = kk < best ? kk : best;
-          }
+#pragma unroll 1
+        for (int l = tid; l < L; l += kConsumers) {
+          if (a.committed[row0 + l] != 0) continue;
+          const float H = __ldcg(a.H_out + row0 + l);
+          if (mi && (double)H <= a.gamma) continue;
+          const unsigned long long kk = key_asc(H, l);
+          best = kk < best ? kk : best;
         }
         best = block_min_u64(best, ctrl, tid);
         if (tid == 0 && best != ~0ull) pick[(int)(best & 0xffffffffu)] = 1;
       }
-    } else {  // block refinement
-      int nmine = 0;
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        const int l = tid + k * kConsumers;
-        if (l < L && openr[k]) {
-          if ((double)pmr[k] >= a.theta) pick[l] = 1;
-          else ++nmine;
-        }
-      }
-      int n_r = 0;
-      int pos = block_excl_scan(nmine, ctrl, tid, &n_r);
-#pragma unroll
-      for (int k = 0; k < kPerThread; ++k) {
-        const int l = tid + k * kConsumers;
-        if (l < L && openr[k] && !((double)pmr[k] >= a.theta)) keys[pos++] = key_desc(pmr[k], l);
-      }
-      consumer_sync(kConsumers);
-      if (a.quota > 0) {
-        for (int c = tid; c < n_r; c += kConsumers) {
-          const unsigned long long kc = keys[c];
-          int rank = 0;
-          for (int j = 0; j < n_r; ++j) rank += keys[j] < kc;
-          if (rank < a.quota) pick[(int)(kc & 0xffffffffu)] = 1;
-        }
-      }
     }
     consumer_sync(kConsumers);
+  }
 
-    int left = 0;
-#pragma unroll
-    for (int k = 0; k < kPerThread; ++k) {
-      const int l = tid + k * kConsumers;
-      if (l < L && openr[k]) {
-        if (pick[l] || last_step) {
-          a.canvas[row0 + l] = a.greedy ? amr[k] : smr[k];
-          a.committed[row0 + l] = 1;
-        } else {
-          ++left;
-          const Words4 r = philox((uint32_t)l >> 2, 0u, (uint32_t)a.s,
-                                  bg | (kStreamRenoise << 24), a.key0, a.key1);
-          a.canvas[row0 + l] = (int32_t)uniform_token(pick_word(r, (uint32_t)l & 3u), (uint32_t)a.V);
-        }
+  // Final pass: commit, renoise, remember the argmax.
+  const uint32_t bg = (uint32_t)(a.canvas_offset + bi);
+  int left = 0;
+#pragma unroll 1
+  for (int l = tid; l < L; l += kConsumers) {
+    const int am = __ldcg(a.amax_out + row0 + l);
+    if (a.committed[row0 + l] == 0) {
+      if (fired) {
+        a.canvas[row0 + l] = am;
+        a.committed[row0 + l] = 1;
+      } else if (pick[l] || last_step) {
+        a.canvas[row0 + l] = a.greedy ? am : __ldcg(a.sample + row0 + l);
+        a.committed[row0 + l] = 1;
+      } else {
+        ++left;
+        const Words4 r = philox((uint32_t)l >> 2, 0u, (uint32_t)a.s, bg | (kStreamRenoise << 24),
+                                a.key0, a.key1);
+        a.canvas[row0 + l] = (int32_t)uniform_token(pick_word(r, (uint32_t)l & 3u), (uint32_t)a.V);
       }
     }
-    const int left_tot = block_sum_int(left, ctrl, tid);
-    reason = last_step ? 3 : (left_tot == 0 ? 2 : 0);
+    a.prev_amax[row0 + l] = am;
   }
-
-#pragma unroll
-  for (int k = 0; k < kPerThread; ++k) {
-    const int l = tid + k * kConsumers;
-    if (l < L) a.prev_amax[row0 + l] = amr[k];
-  }
-  consumer_sync(kConsumers);
+  const int left_tot = block_sum_int(left, ctrl, tid);
   if (tid == 0) {
     a.stable[bi] = stable_new;
-    a.stop_next[bi] = (uint8_t)reason;
+    a.stop_next[bi] = (uint8_t)(fired ? 1 : last_step ? 3 : left_tot == 0 ? 2 : 0);
   }
 }
 
@@ -698,7 +678,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, Ctrl* ctrl, unsigned 
 // row.  Returns (in lane 0) whether this row completed its canvas.
 // ---------------------------------------------------------------------------
 template <int DT>
-__device__ bool row_combine(const StepArgs& a, unsigned long long r, int bi, int l,
+__device__ __noinline__ bool row_combine(const StepArgs a, unsigned long long r, int bi, int l,
                             unsigned long long NG, int lane) {
   const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
   const int G = gridDim.x;
@@ -711,12 +691,12 @@ __device__ bool row_combine(const StepArgs& a, unsigned long long r, int bi, int
     if (range_start(c, NG, G) < range_start(c + 1, NG, G)) {
       const Partial* src = a.partials + grow * (size_t)a.max_segs + (size_t)i;
       Partial q;
-      q.S = __ldcg(&src->S);
-      q.W = __ldcg(&src->W);
       q.zmax = __ldcg(&src->zmax);
-      q.amax = __ldcg(&src->amax);
+      q.agrp = __ldcg(&src->agrp);
       q.Stop = __ldcg(&src->Stop);
       q.Wtop = __ldcg(&src->Wtop);
+      q.Srest = __ldcg(&src->Srest);
+      q.Wrest = __ldcg(&src->Wrest);
       q.gscore = __ldcg(&src->gscore);
       q.gidx = __ldcg(&src->gidx);
       merge(R, q, a.c2);
@@ -726,33 +706,49 @@ __device__ bool row_combine(const StepArgs& a, unsigned long long r, int bi, int
 
   const char* rowp = reinterpret_cast<const char*>(a.logits) + grow * (size_t)a.V * elt_bytes(DT);
   // Exact (f64) recomputation of the group holding the argmax: its fp32 sums
-  // carry the exact-1 term of the maximum and are replaced.
-  const int jt = R.amax / kGroup;
-  double Se = 0.0, We = 0.0;
+  // (Stop, Wtop) carry the maximum's own term, whose rounding would dominate
+  // the entropy of a confident row, and are replaced.
+  // Exact recomputation of the group holding the argmax: its fp32 sums
+  // (Stop, Wtop) carry the maximum's own term, whose rounding would dominate
+  // the entropy of a confident row.  Here every element equal to the maximum
+  // contributes exactly 1 (d = (z - zmax) c2 = 0) and is counted apart from
+  // the smaller terms, which keep full relative precision.
+  const int jt = R.agrp;
+  float ss = 0.f, wsum = 0.f;
+  int nmax = 0;
+  int am = 0x7fffffff;  // lowest index of the maximum (it lies in the top group)
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
     const int v = jt * kGroup + lane + 32 * h;
     if (v < a.V) {
-      const double d = ((double)load_elem<DT>(rowp, v) - (double)R.zmax) * a.c2d;
-      const double p = exp2(d);
-      Se += p;
-      We += p * d;
+      const float z = load_elem<DT>(rowp, v);
+      const float d = (z - R.zmax) * a.c2;
+      if (d == 0.f) {
+        ++nmax;
+        am = min(am, v);
+      } else {
+        const float p = ex2(d);
+        ss += p;
+        wsum = fmaf(p, d, wsum);
+      }
     }
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
-    Se += __shfl_xor_sync(0xffffffffu, Se, o);
-    We += __shfl_xor_sync(0xffffffffu, We, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+    nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
+    am = min(am, __shfl_xor_sync(0xffffffffu, am, o));
   }
-  const double S = R.S - (double)R.Stop + Se;
-  const double W = R.W - (double)R.Wtop + We;
+  const double S = (double)nmax + ((double)ss + (double)R.Srest);
+  const double W = (double)wsum + (double)R.Wrest;
   const double H = log(S) - 0.6931471805599453 * (W / S);
 
   const bool open = a.committed[grow] == 0;
   int smp = -1;
   if (open) {
     if (a.greedy || R.gidx == 0x7fffffff) {
-      smp = R.amax;
+      smp = am;
     } else {
       // Element-level Gumbel-max inside the winning group.
       const uint32_t bg = (uint32_t)(a.canvas_offset + bi);
@@ -786,7 +782,7 @@ __device__ bool row_combine(const StepArgs& a, unsigned long long r, int bi, int
   bool canvas_done = false;
   if (lane == 0) {
     a.H_out[grow] = (float)H;
-    a.amax_out[grow] = R.amax;
+    a.amax_out[grow] = am;
     a.sample[grow] = smp;
     a.pmax[grow] = (float)(1.0 / S);
     if (!isfinite(S) || !isfinite(W)) atomicOr(a.status, kStatusNonFinite);
@@ -905,7 +901,8 @@ __global__ void __launch_bounds__(kThreads, DT == kBF16 ? 4 : 3) step_kernel(con
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
     if (TMA && lane == 0) {
-      TileIter it{g_lo, g_hi, a.ng};
+      const uint64_t policy = evict_first_policy();
+      TileIter it(g_lo, g_hi, a.ng, a.L);
       Tile t;
       int k = 0;
       while (it.next(t)) {
@@ -917,23 +914,21 @@ __global__ void __launch_bounds__(kThreads, DT == kBF16 ? 4 : 3) step_kernel(con
           }
         }
         if (*(volatile int*)&ctrl->abort) break;
-        const int bi = act[t.r / a.L];
-        const int l = (int)(t.r % a.L);
-        const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
+        const size_t grow = (size_t)act[t.ai] * (size_t)a.L + (size_t)t.l;
         const size_t e0 = (size_t)t.j0 * kGroup;
         size_t nel = (size_t)t.cnt * kGroup;
         if (e0 + nel > (size_t)a.V) nel = (size_t)a.V - e0;
         const uint32_t bytes = (uint32_t)(nel * elt_bytes(DT));
         mbar_arrive_expect_tx(&full[st], bytes);
         bulk_load(ring + (size_t)st * tile_bytes(DT), logits + grow * row_bytes + e0 * elt_bytes(DT),
-                  bytes, &full[st]);
+                  bytes, &full[st], policy);
         ++k;
         *(volatile int*)&ctrl->issued = k;
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    TileIter it{g_lo, g_hi, a.ng};
+    TileIter it(g_lo, g_hi, a.ng, a.L);
     Tile t;
     int k = 0;
     long long cur_r = -1;
@@ -950,8 +945,8 @@ __global__ void __launch_bounds__(kThreads, DT == kBF16 ? 4 : 3) step_kernel(con
         cur_r = t.r;
         seg_groups = 0;
         acc = empty_partial();
-        bi = act[t.r / a.L];
-        l = (int)(t.r % a.L);
+        bi = act[t.ai];
+        l = t.l;
         const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
         sampling = !a.greedy && a.committed[grow] == 0;
       }
@@ -974,16 +969,15 @@ __global__ void __launch_bounds__(kThreads, DT == kBF16 ? 4 : 3) step_kernel(con
           const unsigned char* gp =
               ring + (size_t)st * tile_bytes(DT) + (size_t)tid * kGroup * elt_bytes(DT);
           if (glen == kGroup) {
-            gs = DT == kBF16 ? group_bf16_full(gp, rot, a.c2, acc.zmax)
-                             : group_f32_full(gp, rot, a.c2, acc.zmax);
+            gs = DT == kBF16 ? group_bf16_full(gp, rot, a.c2) : group_f32_full(gp, rot, a.c2);
           } else {
-            gs = group_scalar<DT>(gp, glen, a.c2, acc.zmax);
+            gs = group_scalar<DT>(gp, glen, a.c2);
           }
         } else {
           const char* gp = logits + grow * row_bytes + (size_t)j * kGroup * elt_bytes(DT);
-          gs = group_scalar<DT>(gp, glen, a.c2, acc.zmax);
+          gs = group_scalar<DT>(gp, glen, a.c2);
         }
-        fold_group(acc, gs, j * kGroup, a.c2);
+        fold_group(acc, gs, j, a.c2);
         if (sampling) lse = 0.6931471805599453f * fmaf(gs.m, a.c2, lg2(gs.S));
       }
       if (TMA) {
