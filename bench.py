@@ -69,7 +69,7 @@ def peaks():
 
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in ("eb_step.cuh", "eb_device.cuh", "eb_sampler.cu"):
+    for f in ("eb_stream.cuh", "eb_finish.cuh", "eb_common.cuh", "eb_device.cuh", "eb_sampler.cu"):
         with open(os.path.join(ROOT, "entropy_bound_canvas_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -78,7 +78,7 @@ def kernel_source_hash():
 def recorded_traffic():
     """DRAM bytes per launch of the step kernel from the committed ncu summary,
     if it was taken on the current kernel source."""
-    path = os.path.join(ROOT, "profiles", "step_kernel_canvas_1x256x262144_bf16.md")
+    path = os.path.join(ROOT, "profiles", "stream_kernel_canvas_1x256x262144_bf16.md")
     try:
         txt = open(path).read()
     except OSError:
@@ -305,7 +305,8 @@ def run_ours(args):
     torch.cuda.synchronize()
 
     full, rem = divmod(K, N)
-    launches = full * (N + 1) + (rem + (1 if rem else 0))
+    # per step: the stream kernel and the finish kernel; per trajectory: the init kernel
+    launches = full * (2 * N + 1) + (2 * rem + (1 if rem else 0))
     pos_per_traj = sum(active) * w.L
     positions = full * pos_per_traj + sum(active[:rem]) * w.L
     bytes_steps = full * sum(active) + sum(active[:rem])
@@ -415,7 +416,7 @@ def run_ours(args):
             "hbm_frac_of_peak": hbm_gbs_job / (peak * world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "ebk::step_kernel<bf16, bulk-copy>",
+                         "kernel": "ebk::stream_kernel<bf16, bulk-copy> + ebk::finish_kernel<bf16>",
                          "kernel_ms": k_ms, "algorithmic_bytes": k_bytes,
                          "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"},
             "cpu_baseline": cpu,

@@ -11,7 +11,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 SRC = os.path.join(HERE, "csrc", "eb_sampler.cu")
-DEPS = [SRC, os.path.join(HERE, "csrc", "eb_step.cuh"), os.path.join(HERE, "csrc", "eb_device.cuh"),
+DEPS = [SRC, os.path.join(HERE, "csrc", "eb_stream.cuh"), os.path.join(HERE, "csrc", "eb_finish.cuh"),
+        os.path.join(HERE, "csrc", "eb_common.cuh"), os.path.join(HERE, "csrc", "eb_device.cuh"),
         os.path.join(ROOT, "include", "eb_sampler.h")]
 LIB = os.path.join(HERE, "libebsampler.so")
 

@@ -82,6 +82,11 @@ __device__ __forceinline__ float gumbel(uint32_t x) {
   return -0.6931471805599453f * lg2(e);
 }
 
+// 1 - u for the same word, exactly: (2 (~x >> 9) + 1) 2^-24.
+__device__ __forceinline__ float one_minus_u(uint32_t x) {
+  return (float)((~x >> 9) * 2u + 1u) * 5.9604644775390625e-08f;
+}
+
 // Largest Gumbel value the 23-bit grid can produce, -ln(-ln(1 - 2^-24)) =
 // 16.6355..., rounded up; a group whose log-partition plus this bound is
 // below the best score so far cannot win.
@@ -155,6 +160,14 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       "l"(gsrc), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
+
+// Programmatic dependent launch: the dependent grid may be scheduled once
+// every CTA of this grid has signalled (or exited); griddep_wait blocks until
+// the prerequisite grid has completed and its memory operations are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // Named barrier among the consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumer_sync(int nthreads) {

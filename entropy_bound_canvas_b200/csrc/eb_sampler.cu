@@ -1,8 +1,11 @@
 // eb_sampler.cu -- host side of the C ABI declared in include/eb_sampler.h.
 //
-// Validation, the device workspace, launch configuration (one persistent
-// step kernel per call, sized to fill every SM) and error codes.  All the
-// per-step arithmetic runs in the kernels of eb_step.cuh.
+// Validation, the device workspace, launch configuration and error codes.
+// A step is two kernels on the caller's stream: the persistent stream kernel
+// (eb_stream.cuh, sized to fill every SM) and the finish kernel
+// (eb_finish.cuh, one 8-CTA cluster per canvas), launched as a programmatic
+// dependent of the first so that its launch overlaps the first one's end.
+// All the per-step arithmetic runs in those kernels.
 #include "eb_sampler.h"
 
 #include <cuda_runtime.h>
@@ -13,7 +16,8 @@
 #include <cstring>
 #include <new>
 
-#include "eb_step.cuh"
+#include "eb_finish.cuh"
+#include "eb_stream.cuh"
 
 namespace {
 
@@ -34,21 +38,19 @@ struct eb_sampler {
   int sms = 0;
   int ng = 0;
   int max_segs = 0;
-  KernelCfg k[2][2];  // [dtype][tma]
+  KernelCfg k[2][2];  // stream kernel [dtype][tma]
+  KernelCfg fin[2];   // finish kernel [dtype]
   // workspace (one allocation)
   void* ws = nullptr;
   size_t ws_bytes = 0;
   Partial* partials = nullptr;
-  uint32_t* row_ticket = nullptr;
-  uint32_t* canvas_ticket = nullptr;
-  uint32_t* exit_ticket = nullptr;
   uint32_t* status = nullptr;
+  int32_t* act_index = nullptr;
+  int32_t* n_act = nullptr;
   int32_t* prev_amax = nullptr;
   int32_t* stable = nullptr;
   int32_t* sample = nullptr;
   float* pmax = nullptr;
-  uint8_t* stop_next = nullptr;
-  size_t tickets_bytes = 0;  // row + canvas + exit tickets, contiguous
   int last_step = -1;
 };
 
@@ -93,22 +95,36 @@ int validate_config(const eb_config_t* c) {
 template <int DT, bool TMA>
 int setup_kernel(eb_sampler* h, const cudaDeviceProp& prop) {
   KernelCfg& kc = h->k[DT][TMA ? 1 : 0];
-  const ebk::Layout lay = ebk::make_layout(DT, h->cfg.B, h->cfg.L);
-  kc.fn = reinterpret_cast<const void*>(&ebk::step_kernel<DT, TMA>);
+  const ebk::StreamLayout lay = ebk::stream_layout<DT>(h->cfg.B);
+  kc.fn = reinterpret_cast<const void*>(&ebk::stream_kernel<DT, TMA>);
   kc.smem = lay.total;
   if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
-  if (cudaFuncSetAttribute(ebk::step_kernel<DT, TMA>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kc.smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(ebk::stream_kernel<DT, TMA>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kc.smem) != cudaSuccess)
     return EB_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::step_kernel<DT, TMA>,
-                                                    ebk::kThreads, kc.smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::stream_kernel<DT, TMA>,
+                                                    ebk::StreamShape<DT>::kThreads, kc.smem) != cudaSuccess ||
       per_sm < 1)
     return EB_ERR_CUDA;
   const uint64_t groups = (uint64_t)h->cfg.B * (uint64_t)h->cfg.L * (uint64_t)h->ng;
-  const uint64_t want = (groups + ebk::kTileGroups - 1) / ebk::kTileGroups;
+  const uint64_t want =
+      (groups + ebk::StreamShape<DT>::kTileGroups - 1) / ebk::StreamShape<DT>::kTileGroups;
   kc.grid = (int)std::min<uint64_t>((uint64_t)per_sm * (uint64_t)prop.multiProcessorCount,
                                     std::max<uint64_t>(1, want));
+  return EB_OK;
+}
+
+template <int DT>
+int setup_finish(eb_sampler* h, const cudaDeviceProp& prop) {
+  KernelCfg& kc = h->fin[DT];
+  kc.fn = reinterpret_cast<const void*>(&ebk::finish_kernel<DT>);
+  kc.smem = ebk::fin_layout(h->cfg.L).total;
+  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
+  if (cudaFuncSetAttribute(ebk::finish_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kc.smem) != cudaSuccess)
+    return EB_ERR_CUDA;
+  kc.grid = h->cfg.B * ebk::kFinCluster;
   return EB_OK;
 }
 
@@ -160,7 +176,9 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   if ((rc = setup_kernel<ebk::kF32, true>(h, prop)) != EB_OK ||
       (rc = setup_kernel<ebk::kF32, false>(h, prop)) != EB_OK ||
       (rc = setup_kernel<ebk::kBF16, true>(h, prop)) != EB_OK ||
-      (rc = setup_kernel<ebk::kBF16, false>(h, prop)) != EB_OK) {
+      (rc = setup_kernel<ebk::kBF16, false>(h, prop)) != EB_OK ||
+      (rc = setup_finish<ebk::kF32>(h, prop)) != EB_OK ||
+      (rc = setup_finish<ebk::kBF16>(h, prop)) != EB_OK) {
     delete h;
     return rc;
   }
@@ -178,11 +196,10 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   size_t off = 0;
   const size_t o_part = off;
   off = align256(off + sizeof(Partial) * BL * (size_t)h->max_segs);
-  const size_t o_tick = off;
-  h->tickets_bytes = sizeof(uint32_t) * (BL + (size_t)cfg->B + 1);
-  off = align256(off + h->tickets_bytes);
   const size_t o_status = off;
   off = align256(off + sizeof(uint32_t));
+  const size_t o_act = off;
+  off = align256(off + sizeof(int32_t) * ((size_t)cfg->B + 1));
   const size_t o_prev = off;
   off = align256(off + sizeof(int32_t) * BL);
   const size_t o_stable = off;
@@ -191,8 +208,6 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   off = align256(off + sizeof(int32_t) * BL);
   const size_t o_pmax = off;
   off = align256(off + sizeof(float) * BL);
-  const size_t o_stopn = off;
-  off = align256(off + (size_t)cfg->B);
   h->ws_bytes = off;
   if (cudaMalloc(&h->ws, h->ws_bytes) != cudaSuccess) {
     cudaGetLastError();
@@ -206,15 +221,13 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   }
   char* base = static_cast<char*>(h->ws);
   h->partials = reinterpret_cast<Partial*>(base + o_part);
-  h->row_ticket = reinterpret_cast<uint32_t*>(base + o_tick);
-  h->canvas_ticket = h->row_ticket + BL;
-  h->exit_ticket = h->canvas_ticket + cfg->B;
   h->status = reinterpret_cast<uint32_t*>(base + o_status);
+  h->act_index = reinterpret_cast<int32_t*>(base + o_act);
+  h->n_act = h->act_index + cfg->B;
   h->prev_amax = reinterpret_cast<int32_t*>(base + o_prev);
   h->stable = reinterpret_cast<int32_t*>(base + o_stable);
   h->sample = reinterpret_cast<int32_t*>(base + o_sample);
   h->pmax = reinterpret_cast<float*>(base + o_pmax);
-  h->stop_next = reinterpret_cast<uint8_t*>(base + o_stopn);
   *out = h;
   return EB_OK;
 }
@@ -226,7 +239,7 @@ int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
   if (!guard.ok) return EB_ERR_CUDA;
   const eb_config_t& c = h->cfg;
   ebk::init_canvas_kernel<<<c.B, 256, 0, (cudaStream_t)stream>>>(
-      canvas, committed, stop_flags, h->stable, h->stop_next, c.L, c.V, c.canvas_offset,
+      canvas, committed, stop_flags, h->stable, c.L, c.V, c.canvas_offset,
       (uint32_t)(c.seed & 0xffffffffu), (uint32_t)(c.seed >> 32));
   if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = -1;
@@ -246,10 +259,6 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   if (!guard.ok) return EB_ERR_CUDA;
   cudaStream_t st = (cudaStream_t)stream;
 
-  if (step == 0) {  // tickets are self-resetting; clear them anyway at a restart
-    if (cudaMemsetAsync(h->row_ticket, 0, h->tickets_bytes, st) != cudaSuccess) return EB_ERR_CUDA;
-  }
-
   const double T = c.greedy ? 1.0
                    : c.num_steps <= 1
                        ? c.t_max
@@ -263,15 +272,13 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.amax_out = argmax;
   a.stop_flags = stop_flags;
   a.partials = h->partials;
-  a.row_ticket = h->row_ticket;
-  a.canvas_ticket = h->canvas_ticket;
-  a.exit_ticket = h->exit_ticket;
   a.prev_amax = h->prev_amax;
   a.stable = h->stable;
   a.sample = h->sample;
   a.pmax = h->pmax;
-  a.stop_next = h->stop_next;
   a.status = h->status;
+  a.act_index = h->act_index;
+  a.n_act = h->n_act;
   a.B = c.B;
   a.L = c.L;
   a.V = c.V;
@@ -296,10 +303,29 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   const size_t elt = dtype == EB_F32 ? 4 : 2;
   const bool tma = ((uintptr_t)logits % 16 == 0) && (((size_t)c.V * elt) % 16 == 0);
   const KernelCfg& kc = h->k[dtype][tma ? 1 : 0];
+  a.G1 = kc.grid;
+  a.vec_ok = tma ? 1 : 0;
   void* args[] = {&a};
-  if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::kThreads), args, kc.smem, st) !=
+  if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), args, kc.smem, st) !=
       cudaSuccess)
     return EB_ERR_CUDA;
+
+  const KernelCfg& kf = h->fin[dtype];
+  const int32_t* act_index = h->act_index;
+  const int32_t* n_act = h->n_act;
+  void* fargs[] = {&a, &act_index, &n_act};
+  cudaLaunchConfig_t lc;
+  std::memset(&lc, 0, sizeof(lc));
+  lc.gridDim = dim3(kf.grid);
+  lc.blockDim = dim3(ebk::kFinThreads);
+  lc.dynamicSmemBytes = kf.smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  if (cudaLaunchKernelExC(&lc, kf.fn, fargs) != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = step;
   return EB_OK;
 }
@@ -385,7 +411,6 @@ int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int3
              cudaSuccess) {
     return EB_ERR_CUDA;
   }
-  if (cudaMemsetAsync(h->row_ticket, 0, h->tickets_bytes, st) != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = next_step - 1;
   return EB_OK;
 }
