@@ -55,9 +55,11 @@ struct StepArgs {
   uint32_t* status;
   int32_t* act_index;  // [B] written by the stream kernel: active index or -1
   int32_t* n_act;      // [1] written by the stream kernel
-  int B, L, V, ng, s, N, max_segs;
-  int G1;      // grid size of the stream kernel (its group split)
-  int vec_ok;  // rows start on 16-byte boundaries (vector loads allowed)
+  int B, L, V, ng, s, N;
+  int max_segs;  // stream CTAs that can share one row
+  int nw;        // Partial records per (row, stream CTA): its consumer warps
+  int G1;        // grid size of the stream kernel (its group split)
+  int vec_ok;    // rows start on 16-byte boundaries (vector loads allowed)
   int rule, quota, stability_steps, greedy, stop_enabled;
   int canvas_offset;
   float c2, iT;
@@ -154,12 +156,6 @@ __device__ __forceinline__ void warp_merge(Partial& p, float c2) {
 // ---------------------------------------------------------------------------
 // Packed arithmetic and group reductions
 // ---------------------------------------------------------------------------
-struct GroupStat {
-  float m;  // raw maximum
-  float S;  // sum 2^d, d = (z - m) c2
-  float W;  // sum 2^d d
-};
-
 // Lane-wise maximum of two packed bf16 pairs.
 __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -186,9 +182,9 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return r;
 }
 
-// One pair of logits: d = z c2 - m c2, p = 2^d, S += p, W += p d.  The
-// maximum itself gets d = the rounding residue of m c2 rather than 0; the
-// finish kernel recomputes the group holding the argmax exactly.
+// One pair of logits: d = z c2 - r c2, p = 2^d, S += p, W += p d.  An element
+// equal to the reference r gets d = the rounding residue of r c2 rather than
+// 0; the finish kernel recomputes the group holding the row maximum exactly.
 __device__ __forceinline__ void acc_pair(float2 z, float2 c2v, float2 nmc, float2& S, float2& W) {
   const float2 d = ffma2(z, c2v, nmc);
   float2 p;
@@ -198,10 +194,6 @@ __device__ __forceinline__ void acc_pair(float2 z, float2 c2v, float2 nmc, float
   W = ffma2(p, d, W);
 }
 
-__device__ __forceinline__ float tree8(const float (&v)[8]) {
-  return ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
-}
-
 __device__ __forceinline__ float sum4(const float2 (&v)[4]) {
   return ((v[0].x + v[0].y) + (v[1].x + v[1].y)) + ((v[2].x + v[2].y) + (v[3].x + v[3].y));
 }
@@ -209,81 +201,112 @@ __device__ __forceinline__ float sum4(const float2 (&v)[4]) {
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 
-// Full 64-element bf16 group in shared memory (128 bytes), read twice (max,
-// then exponentials) to keep register use low.  Pieces of 16 bytes are read
-// in an order rotated by the thread index so that the eight threads of a
-// shared-memory phase hit eight different bank quads.
-__device__ __forceinline__ GroupStat group_bf16_full(const unsigned char* gp, int rot, float c2) {
-  const uint4* q = reinterpret_cast<const uint4*>(gp);
-  uint32_t mx0, mx1;
-  {
-    const uint4 v = q[rot & 7];
-    mx0 = bf16x2_max(v.x, v.y);
-    mx1 = bf16x2_max(v.z, v.w);
-  }
-#pragma unroll
-  for (int k = 1; k < 8; ++k) {
-    const uint4 v = q[(k + rot) & 7];
-    mx0 = bf16x2_max(mx0, bf16x2_max(v.x, v.y));
-    mx1 = bf16x2_max(mx1, bf16x2_max(v.z, v.w));
-  }
-  const uint32_t mx = bf16x2_max(mx0, mx1);
-  const float m = fmaxf(bf16_lo(mx), bf16_hi(mx));
-  const float2 c2v = make_float2(c2, c2);
-  const float2 nmc = make_float2(-m * c2, -m * c2);
+// ---------------------------------------------------------------------------
+// Group reductions.  A consumer lane reduces whole 64-logit groups that sit in
+// shared memory.  Max pass: the raw group maximum m_g.  Exponential pass,
+// relative to a reference Mref >= m_g: S_g = sum 2^d, W_g = sum 2^d d with
+// d = (z - Mref) c2.  Pieces of 16 bytes are read in an order rotated by the
+// lane index, so the eight lanes of a shared-memory phase hit eight different
+// bank quads.
+// ---------------------------------------------------------------------------
+template <int DT>
+struct GroupIO;
 
-  float2 S[4], W[4];
+template <>
+struct GroupIO<kBF16> {
+  static constexpr int kPieces = 8;  // 16-byte pieces per group
+  __device__ __forceinline__ static float max_of(const unsigned char* gp, int rot) {
+    const uint4* q = reinterpret_cast<const uint4*>(gp);
+    uint32_t t[16];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    S[i] = make_float2(0.f, 0.f);
-    W[i] = make_float2(0.f, 0.f);
+    for (int k = 0; k < 8; ++k) {
+      const uint4 v = q[(k + rot) & 7];
+      t[2 * k] = bf16x2_max(v.x, v.y);
+      t[2 * k + 1] = bf16x2_max(v.z, v.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t[i] = bf16x2_max(t[2 * i], t[2 * i + 1]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) t[i] = bf16x2_max(t[2 * i], t[2 * i + 1]);
+    const uint32_t m = bf16x2_max(bf16x2_max(t[0], t[1]), bf16x2_max(t[2], t[3]));
+    return fmaxf(bf16_lo(m), bf16_hi(m));
   }
+  // Exponential pass of two groups at once (independent chains interleave).
+  __device__ __forceinline__ static void exp2_of(const unsigned char* g0, const unsigned char* g1,
+                                                 int rot, float c2, float r0, float r1,
+                                                 float& S0, float& W0, float& S1, float& W1) {
+    const uint4* q0 = reinterpret_cast<const uint4*>(g0);
+    const uint4* q1 = reinterpret_cast<const uint4*>(g1);
+    const float2 c2v = make_float2(c2, c2);
+    const float2 n0 = make_float2(-r0 * c2, -r0 * c2), n1 = make_float2(-r1 * c2, -r1 * c2);
+    float2 s0[4], w0[4], s1[4], w1[4];
 #pragma unroll
-  for (int k = 0; k < 8; ++k) {
-    const uint4 v = q[(k + rot) & 7];
-    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 4; ++i) {
+      s0[i] = w0[i] = s1[i] = w1[i] = make_float2(0.f, 0.f);
+    }
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
-      acc_pair(make_float2(bf16_lo(w4[i]), bf16_hi(w4[i])), c2v, nmc, S[i], W[i]);
+    for (int k = 0; k < 8; ++k) {
+      const uint4 a = q0[(k + rot) & 7];
+      const uint4 b = q1[(k + rot) & 7];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+      const uint32_t wb[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        acc_pair(make_float2(bf16_lo(wa[i]), bf16_hi(wa[i])), c2v, n0, s0[i], w0[i]);
+        acc_pair(make_float2(bf16_lo(wb[i]), bf16_hi(wb[i])), c2v, n1, s1[i], w1[i]);
+      }
+    }
+    S0 = sum4(s0);
+    W0 = sum4(w0);
+    S1 = sum4(s1);
+    W1 = sum4(w1);
   }
-  GroupStat g;
-  g.m = m;
-  g.S = sum4(S);
-  g.W = sum4(W);
-  return g;
-}
+};
 
-// Full 64-element fp32 group in shared memory (256 bytes), read twice.
-__device__ __forceinline__ GroupStat group_f32_full(const unsigned char* gp, int rot, float c2) {
-  const float4* q = reinterpret_cast<const float4*>(gp);
-  float m0 = -INFINITY, m1 = -INFINITY;
+template <>
+struct GroupIO<kF32> {
+  static constexpr int kPieces = 16;
+  __device__ __forceinline__ static float max_of(const unsigned char* gp, int rot) {
+    const float4* q = reinterpret_cast<const float4*>(gp);
+    float t[16];
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float4 v = q[(k + rot) & 15];
-    m0 = fmaxf(m0, fmaxf(v.x, v.y));
-    m1 = fmaxf(m1, fmaxf(v.z, v.w));
-  }
-  const float m = fmaxf(m0, m1);
-  const float2 c2v = make_float2(c2, c2);
-  const float2 nmc = make_float2(-m * c2, -m * c2);
-  float2 S[4], W[4];
+    for (int k = 0; k < 16; ++k) {
+      const float4 v = q[(k + rot) & 15];
+      t[k] = fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w));
+    }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    S[i] = make_float2(0.f, 0.f);
-    W[i] = make_float2(0.f, 0.f);
-  }
+    for (int i = 0; i < 8; ++i) t[i] = fmaxf(t[2 * i], t[2 * i + 1]);
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    const float4 v = q[(k + rot) & 15];
-    acc_pair(make_float2(v.x, v.y), c2v, nmc, S[(2 * k) & 3], W[(2 * k) & 3]);
-    acc_pair(make_float2(v.z, v.w), c2v, nmc, S[(2 * k + 1) & 3], W[(2 * k + 1) & 3]);
+    for (int i = 0; i < 4; ++i) t[i] = fmaxf(t[2 * i], t[2 * i + 1]);
+    return fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3]));
   }
-  GroupStat g;
-  g.m = m;
-  g.S = sum4(S);
-  g.W = sum4(W);
-  return g;
-}
+  __device__ __forceinline__ static void exp2_of(const unsigned char* g0, const unsigned char* g1,
+                                                 int rot, float c2, float r0, float r1,
+                                                 float& S0, float& W0, float& S1, float& W1) {
+    const float4* q0 = reinterpret_cast<const float4*>(g0);
+    const float4* q1 = reinterpret_cast<const float4*>(g1);
+    const float2 c2v = make_float2(c2, c2);
+    const float2 n0 = make_float2(-r0 * c2, -r0 * c2), n1 = make_float2(-r1 * c2, -r1 * c2);
+    float2 s0[2], w0[2], s1[2], w1[2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      s0[i] = w0[i] = s1[i] = w1[i] = make_float2(0.f, 0.f);
+    }
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float4 a = q0[(k + rot) & 15];
+      const float4 b = q1[(k + rot) & 15];
+      acc_pair(make_float2(a.x, a.y), c2v, n0, s0[0], w0[0]);
+      acc_pair(make_float2(a.z, a.w), c2v, n0, s0[1], w0[1]);
+      acc_pair(make_float2(b.x, b.y), c2v, n1, s1[0], w1[0]);
+      acc_pair(make_float2(b.z, b.w), c2v, n1, s1[1], w1[1]);
+    }
+    S0 = (s0[0].x + s0[0].y) + (s0[1].x + s0[1].y);
+    W0 = (w0[0].x + w0[0].y) + (w0[1].x + w0[1].y);
+    S1 = (s1[0].x + s1[0].y) + (s1[1].x + s1[1].y);
+    W1 = (w1[0].x + w1[0].y) + (w1[1].x + w1[1].y);
+  }
+};
 
 template <int DT>
 __device__ __forceinline__ float load_elem(const void* p, int e) {
@@ -291,54 +314,149 @@ __device__ __forceinline__ float load_elem(const void* p, int e) {
   return __uint_as_float((uint32_t) reinterpret_cast<const uint16_t*>(p)[e] << 16);
 }
 
-// Any group (partial last group of a row, or unaligned rows): element by
-// element through a generic pointer (shared or global memory).
+// Any group element by element (a partial last group of a row, rows that are
+// not 16-byte aligned, or a group whose fast-path sums were not finite).
 template <int DT>
-__device__ __noinline__ GroupStat group_scalar(const void* gp, int glen, float c2) {
+__device__ __noinline__ float group_max_safe(const void* gp, int glen) {
   float m = -INFINITY;
   for (int e = 0; e < glen; ++e) m = fmaxf(m, load_elem<DT>(gp, e));
-  float s[8], ws[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    s[i] = 0.f;
-    ws[i] = 0.f;
-  }
-  for (int e = 0; e < glen; ++e) {
-    const float d = (load_elem<DT>(gp, e) - m) * c2;
-    const float p = ex2(d);
-    s[e & 7] += p;
-    ws[e & 7] = fmaf(p, d, ws[e & 7]);
-  }
-  GroupStat g;
-  g.m = m;
-  g.S = tree8(s);
-  g.W = tree8(ws);
-  return g;
+  return m;
 }
 
-// Fold one group into a thread's running partial (a thread sees the groups
-// of a row segment in increasing index order, so a tie never moves the
-// maximum's group).
-__device__ __forceinline__ void fold_group(Partial& t, const GroupStat& g, int j, float c2) {
-  if (g.m > t.zmax) {
-    if (t.zmax > -INFINITY) {
-      const float d = (t.zmax - g.m) * c2;
-      const float f = ex2(d);
-      const float S = t.Stop + t.Srest;
-      const float W = t.Wtop + t.Wrest;
-      t.Srest = f * S;
-      t.Wrest = f * fmaf(d, S, W);
+// Sums relative to the reference r over the elements whose term is nonzero,
+// so that a -inf logit contributes nothing (rather than 0 * -inf).
+template <int DT>
+__device__ __noinline__ float2 group_sums_safe(const void* gp, int glen, float c2, float r) {
+  float S = 0.f, W = 0.f;
+  if (r > -INFINITY) {
+    for (int e = 0; e < glen; ++e) {
+      const float d = (load_elem<DT>(gp, e) - r) * c2;
+      const float p = ex2(d);
+      if (p > 0.f) {
+        S += p;
+        W = fmaf(p, d, W);
+      }
     }
-    t.Stop = g.S;
-    t.Wtop = g.W;
-    t.zmax = g.m;
-    t.agrp = j;
-  } else {
-    const float d = (g.m - t.zmax) * c2;
-    const float f = ex2(d);
-    t.Srest = fmaf(f, g.S, t.Srest);
-    t.Wrest = fmaf(f, fmaf(d, g.S, g.W), t.Wrest);
   }
+  return make_float2(S, W);
+}
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ int warp_min_i(int v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Running state of one warp over the groups of one row segment.  Every lane
+// holds the same M (largest logit so far), tgrp (lowest group holding M), R
+// (best Gumbel ratio) and gbest (its group); each lane holds its own sums,
+// relative to M, of the groups it reduced: those of group tgrp (top) apart
+// from all others (rest).  Group j's Gumbel-perturbed log-partition is
+// ln Z_j + M / T - ln E_j, with Z_j its S relative to M and E_j = -ln u_j, so
+// the winning group is the one with the largest ratio Z_j / E_j.
+struct WarpAcc {
+  float M, R;
+  int tgrp, gbest;
+  float Stop, Wtop, Srest, Wrest;
+};
+
+__device__ __forceinline__ void warp_reset(WarpAcc& A) {
+  A.M = -INFINITY;
+  A.R = 0.f;
+  A.tgrp = 0x7fffffff;
+  A.gbest = 0x7fffffff;
+  A.Stop = A.Wtop = A.Srest = A.Wrest = 0.f;
+}
+
+// Before the exponential pass of a sub-tile: this lane's largest group
+// maximum m_loc (first reached at group j_loc) joins the warp's M.  On a new
+// maximum every sum (and R) is rescaled to it, the old top group joins the
+// rest, and the lowest group holding the new maximum becomes the top group.
+__device__ __forceinline__ void warp_raise(WarpAcc& A, float m_loc, int j_loc, float c2) {
+  const float Mn = warp_max_f(fmaxf(A.M, m_loc));
+  if (Mn > A.M) {  // warp-uniform
+    if (A.M > -INFINITY) {
+      const float dd = (A.M - Mn) * c2;
+      const float f = ex2(dd);
+      const float S = A.Stop + A.Srest;
+      const float W = A.Wtop + A.Wrest;
+      A.Srest = f * S;
+      A.Wrest = f * fmaf(dd, S, W);
+      A.R *= f;
+    }
+    A.Stop = A.Wtop = 0.f;
+    A.M = Mn;
+    A.tgrp = warp_min_i(m_loc == Mn ? j_loc : 0x7fffffff);
+  }
+}
+
+// One group's sums (relative to M) into the lane's top or rest.
+__device__ __forceinline__ void warp_fold(WarpAcc& A, float S, float W, int j) {
+  if (j == A.tgrp) {
+    A.Stop = S;
+    A.Wtop = W;
+  } else {
+    A.Srest += S;
+    A.Wrest += W;
+  }
+}
+
+// Gumbel race of one group (Z = its S relative to M, group-stream word x)
+// against the lane's running best (Rl, gl), which starts at the warp's R.
+// Since E = -ln u >= 1 - u, a group with Z <= R (1 - u) cannot beat R
+// (checked with a 1e-4 relative margin): its logarithm is skipped.
+__device__ __forceinline__ void lane_race(float& Rl, int& gl, float Z, uint32_t x, int j) {
+  if (Z * 1.0001f <= Rl * one_minus_u(x)) return;
+  const float E = -logf(uniform_open(x));
+  if (Z > Rl * E) {
+    Rl = __fdividef(Z, E);
+    gl = j;
+  }
+}
+
+// After the race of a sub-tile: the warp's best ratio (ties: lower group).
+__device__ __forceinline__ void warp_race_merge(WarpAcc& A, float Rl, int gl) {
+  if (!__any_sync(0xffffffffu, gl != 0x7fffffff)) return;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float oR = __shfl_xor_sync(0xffffffffu, Rl, o);
+    const int og = __shfl_xor_sync(0xffffffffu, gl, o);
+    if (oR > Rl || (oR == Rl && og < gl)) {
+      Rl = oR;
+      gl = og;
+    }
+  }
+  A.R = Rl;
+  A.gbest = gl;
+}
+
+// The warp's state as one Partial record (absolute Gumbel score ln R + M/T).
+__device__ __forceinline__ Partial warp_record(const WarpAcc& A, float iT) {
+  Partial p;
+  p.zmax = A.M;
+  p.agrp = A.tgrp;
+  p.Stop = warp_sum_f(A.Stop);
+  p.Wtop = warp_sum_f(A.Wtop);
+  p.Srest = warp_sum_f(A.Srest);
+  p.Wrest = warp_sum_f(A.Wrest);
+  if (A.R > 0.f && A.M > -INFINITY) {
+    p.gscore = fmaf(A.M, iT, logf(A.R));
+    p.gidx = A.gbest;
+  } else {
+    p.gscore = -INFINITY;
+    p.gidx = 0x7fffffff;
+  }
+  return p;
 }
 
 }  // namespace ebk

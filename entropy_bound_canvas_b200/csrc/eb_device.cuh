@@ -73,18 +73,24 @@ __device__ __forceinline__ uint32_t pick_word(const Words4& r, uint32_t i) {
 // Streams of the counter layout: ctr = (index >> 2, a, step, b | stream << 24).
 enum : uint32_t { kStreamGumbel = 0, kStreamRenoise = 1, kStreamInit = 2, kStreamGroup = 3 };
 
-// Standard Gumbel from one word: u = (2 (x >> 9) + 1) 2^-24 (exact in fp32),
-// g = -ln(-ln u).  The inner log must be accurate near u = 1 (logf, ~1 ulp);
-// the outer one only needs absolute accuracy, which lg2.approx gives.
-__device__ __forceinline__ float gumbel(uint32_t x) {
-  const float u = (float)((x >> 9) * 2u + 1u) * 5.9604644775390625e-08f;
-  const float e = -logf(u);
-  return -0.6931471805599453f * lg2(e);
+// The uniform of a word x: u = (2 (x >> 9) + 1) 2^-24, in (0, 1), built
+// exactly from bits: 1 + (x >> 9) 2^-23 lies in [1, 2), and subtracting
+// 1 - 2^-24 is exact (both operands within a factor of two).
+__device__ __forceinline__ float uniform_open(uint32_t x) {
+  return __uint_as_float(0x3F800000u | (x >> 9)) - 0.99999994039535522f;
 }
 
 // 1 - u for the same word, exactly: (2 (~x >> 9) + 1) 2^-24.
 __device__ __forceinline__ float one_minus_u(uint32_t x) {
-  return (float)((~x >> 9) * 2u + 1u) * 5.9604644775390625e-08f;
+  return __uint_as_float(0x3F800000u | (~x >> 9)) - 0.99999994039535522f;
+}
+
+// Standard Gumbel from one word: g = -ln(-ln u).  The inner log must be
+// accurate near u = 1 (logf, ~1 ulp); the outer one only needs absolute
+// accuracy, which lg2.approx gives.
+__device__ __forceinline__ float gumbel(uint32_t x) {
+  const float e = -logf(uniform_open(x));
+  return -0.6931471805599453f * lg2(e);
 }
 
 // Largest Gumbel value the 23-bit grid can produce, -ln(-ln(1 - 2^-24)) =
@@ -140,6 +146,30 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (global_ns() - t0 > kWaitLimitNs) return false;
+  }
+}
+
+// Shared-memory counter published by one thread and polled by others.
+__device__ __forceinline__ void st_release_shared(int* p, int v) {
+  asm volatile("st.release.cta.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v) : "memory");
+}
+__device__ __forceinline__ int ld_acquire_shared(const int* p) {
+  int v;
+  asm volatile("ld.acquire.cta.shared::cta.b32 %0, [%1];" : "=r"(v) : "r"(smem_u32(p)) : "memory");
+  return v;
+}
+
+// Waits (bounded like mbar_wait) until *p > k.
+__device__ __forceinline__ bool wait_counter_above(const int* p, int k) {
+  if (ld_acquire_shared(p) > k) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      __nanosleep(32);
+      if (ld_acquire_shared(p) > k) return true;
+    }
     if (global_ns() - t0 > kWaitLimitNs) return false;
   }
 }

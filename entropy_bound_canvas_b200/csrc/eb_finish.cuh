@@ -12,8 +12,8 @@
 //      group (element-stream Philox words; the element with the largest
 //      logit is drawn first and the logarithms of every element that cannot
 //      beat it are skipped exactly),
-// then the cluster synchronises and rank 0 gathers the slice results from its
-// peers' shared memory and runs the canvas epilogue: argmax stability,
+// and writes its results straight into cluster rank 0's shared memory; after
+// one cluster barrier rank 0 runs the canvas epilogue: argmax stability,
 // adaptive stop, commit rule, last-step / all-committed finalisation and
 // renoise.  Only hardware barriers (CTA and cluster) are used.
 //
@@ -41,14 +41,14 @@ constexpr int kFinWarps = kFinThreads / 32;
 
 struct FinCtrl {
   int kpref;
-  int pad;
+  int stable_prev;
   double dscr[kFinWarps];
   int iscr[kFinWarps];
   unsigned long long uscr[kFinWarps];
 };
 
 struct FinLayout {
-  uint32_t ctrl, H, am, smp, pm, open, pick, keys, skeys, total;
+  uint32_t ctrl, H, am, smp, pm, prev, tok, open, pick, keys, skeys, total;
 };
 
 __host__ __device__ inline FinLayout fin_layout(int L) {
@@ -68,6 +68,10 @@ __host__ __device__ inline FinLayout fin_layout(int L) {
   y.smp = o;
   o += 4u * l;
   y.pm = o;
+  o += 4u * l;
+  y.prev = o;
+  o += 4u * l;
+  y.tok = o;
   o += 4u * l;
   y.open = o;
   o += l;
@@ -161,7 +165,7 @@ __device__ __forceinline__ unsigned long long key_desc(float p, int l) {
 }
 
 // ---------------------------------------------------------------------------
-// Per-position work of one subgroup of `tpr` lanes (all lanes of a warp
+// Per-position work of one subgroup of TPR lanes (all lanes of a warp
 // execute it; `valid` is false for lanes without a position).
 // ---------------------------------------------------------------------------
 struct RowOut {
@@ -169,54 +173,116 @@ struct RowOut {
   int amax, sample;
 };
 
-template <int DT>
+// The PER logits v0 .. v0 + PER - 1 of one row (those >= V read as -inf):
+// vector loads when the row is 16-byte aligned and the chunk is whole.
+template <int DT, int PER>
+__device__ __forceinline__ void load_chunk(const char* rowp, int v0, int V, bool vec, float (&z)[PER]) {
+  constexpr int kBytes = PER * elt_bytes(DT);
+  const char* p = rowp + (size_t)v0 * elt_bytes(DT);
+  if (vec && v0 + PER <= V && kBytes >= 4) {
+    uint32_t w[kBytes / 4];
+    if constexpr (kBytes >= 16) {
+#pragma unroll
+      for (int i = 0; i < kBytes / 16; ++i) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(p) + i);
+        w[4 * i] = q.x;
+        w[4 * i + 1] = q.y;
+        w[4 * i + 2] = q.z;
+        w[4 * i + 3] = q.w;
+      }
+    } else if constexpr (kBytes == 8) {
+      const uint2 q = __ldg(reinterpret_cast<const uint2*>(p));
+      w[0] = q.x;
+      w[1] = q.y;
+    } else {
+      w[0] = __ldg(reinterpret_cast<const uint32_t*>(p));
+    }
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      if (DT == kF32) {
+        z[e] = __uint_as_float(w[e]);
+      } else {
+        z[e] = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) z[e] = v0 + e < V ? load_elem<DT>(rowp, v0 + e) : -INFINITY;
+  }
+}
+
+template <int DT, int TPR>
 __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, int l, bool valid,
-                                             int tpr, int sl, unsigned long long NG) {
+                                             bool open, int sl, unsigned long long NG) {
+  constexpr int PER = kGroup / TPR;  // elements of a group per lane
   RowOut out;
   const size_t grow = (size_t)bi * (size_t)a.L + (size_t)(valid ? l : 0);
-  // 1. merge the row's partials
+  // 1. merge the row's records: (stream CTAs that own part of the row) x nw
   Partial R = empty_partial();
   if (valid) {
     const unsigned long long r = (unsigned long long)ai * (unsigned long long)a.L + (unsigned long long)l;
     const unsigned long long g_first = r * (unsigned long long)a.ng;
     const int c_first = cta_of(g_first, NG, a.G1);
     const int c_last = cta_of(g_first + (unsigned long long)a.ng - 1ull, NG, a.G1);
-    for (int i = sl; i <= c_last - c_first; i += tpr) {
-      const int c = c_first + i;
-      if (range_start(c, NG, a.G1) < range_start(c + 1, NG, a.G1))
-        merge(R, a.partials[grow * (size_t)a.max_segs + (size_t)i], a.c2);
+    const int nrec = (c_last - c_first + 1) * a.nw;
+    const Partial* rec = a.partials + grow * (size_t)(a.max_segs * a.nw);
+    for (int i = sl; i < nrec; i += TPR) {
+      const int c = c_first + i / a.nw;
+      if (range_start(c, NG, a.G1) < range_start(c + 1, NG, a.G1)) merge(R, rec[i], a.c2);
     }
   }
-  for (int o = 1; o < tpr; o <<= 1) {
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) {
     Partial q = shfl_partial(R, o);
     merge(R, q, a.c2);
   }
 
+  // 2. the lane's slices of the group holding the maximum and of the winning
+  //    Gumbel group, loaded together
   const char* rowp = reinterpret_cast<const char*>(a.logits) + grow * (size_t)a.V * elt_bytes(DT);
-  const int per = kGroup / tpr;  // elements of a group per lane
-  // 2. exact recomputation of the top group
+  const bool has_top = valid && R.agrp != 0x7fffffff;
+  const bool draw = open && !a.greedy && R.gidx != 0x7fffffff;
+  const int vt0 = (has_top ? R.agrp : 0) * kGroup + sl * PER;
+  const int vs0 = (draw ? R.gidx : 0) * kGroup + sl * PER;
+  float zt[PER], zs[PER];
+  if (has_top) load_chunk<DT, PER>(rowp, vt0, a.V, a.vec_ok != 0, zt);
+  if (draw) load_chunk<DT, PER>(rowp, vs0, a.V, a.vec_ok != 0, zs);
+  // element-stream words of the sample slice (independent of the loads)
+  constexpr int NC = PER >= 4 ? PER / 4 : 1;
+  uint32_t xw[NC * 4];
+  const uint32_t c3 = (uint32_t)(a.canvas_offset + bi) | (kStreamGumbel << 24);
+  if (draw) {
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      const Words4 w = philox(((uint32_t)vs0 >> 2) + (uint32_t)c, (uint32_t)l, (uint32_t)a.s, c3,
+                              a.key0, a.key1);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) xw[4 * c + q] = w.w[q];
+    }
+  }
+
+  // 3. exact recomputation of the top group: an element equal to the
+  //    maximum contributes exactly 1, the others 2^d (-inf logits nothing)
   float ss = 0.f, wsum = 0.f;
   int nmax = 0, am = 0x7fffffff;
-  if (valid && R.agrp != 0x7fffffff) {
-    const int e0 = R.agrp * kGroup + sl * per;
-#pragma unroll 4
-    for (int e = 0; e < per; ++e) {
-      const int v = e0 + e;
-      if (v < a.V) {
-        const float z = load_elem<DT>(rowp, v);
-        const float d = (z - R.zmax) * a.c2;
-        if (d == 0.f) {
-          ++nmax;
-          am = min(am, v);
-        } else {
-          const float p = ex2(d);
+  if (has_top) {
+#pragma unroll
+    for (int e = 0; e < PER; ++e) {
+      const float d = (zt[e] - R.zmax) * a.c2;
+      if (d == 0.f) {
+        ++nmax;
+        am = min(am, vt0 + e);
+      } else {
+        const float p = ex2(d);
+        if (p > 0.f) {
           ss += p;
           wsum = fmaf(p, d, wsum);
         }
       }
     }
   }
-  for (int o = 1; o < tpr; o <<= 1) {
+#pragma unroll
+  for (int o = 1; o < TPR; o <<= 1) {
     ss += __shfl_xor_sync(0xffffffffu, ss, o);
     wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
     nmax += __shfl_xor_sync(0xffffffffu, nmax, o);
@@ -227,58 +293,62 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
   out.H = (float)(log(S) - 0.6931471805599453 * (W / S));
   out.pmax = (float)(1.0 / S);
   out.amax = am;
-  if (valid && (!isfinite(S) || !isfinite(W))) atomicOr(a.status, kStatusNonFinite);
+  if (valid && (!isfinite(S) || !isfinite(W) || am == 0x7fffffff))
+    atomicOr(a.status, kStatusNonFinite);
 
-  // 3. the categorical draw of an open position
-  const bool open = valid && a.committed[grow] == 0;
-  const bool draw = open && !a.greedy && R.gidx != 0x7fffffff;
+  // 4. the categorical draw within the winning group: the largest tempered
+  //    logit is drawn first; the logarithms of every element that cannot
+  //    beat it are skipped exactly
   out.sample = open ? am : -1;
   if (__any_sync(0xffffffffu, draw)) {
-    const int jg = draw ? R.gidx : 0;
-    const int e0 = jg * kGroup + sl * per;
-    // largest tempered logit of the group and its lowest index
     float ymax = -INFINITY;
-    int vmax = 0x7fffffff;
+    int emax = -1;
     if (draw) {
-      for (int e = 0; e < per; ++e) {
-        const int v = e0 + e;
-        if (v < a.V) {
-          const float y = load_elem<DT>(rowp, v) * a.iT;
-          if (y > ymax) {
-            ymax = y;
-            vmax = v;
-          }
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const float y = zs[e] * a.iT;
+        if (y > ymax) {
+          ymax = y;
+          emax = e;
         }
       }
     }
-    for (int o = 1; o < tpr; o <<= 1) {
+    // word of element e of the slice (PER >= 4: slices start on a call)
+    auto word_at = [&](int e) -> uint32_t {
+      if constexpr (PER >= 4) {
+        return xw[e];
+      } else {
+        return (vs0 & 2) ? xw[2 + e] : xw[e];
+      }
+    };
+    int vmax = emax >= 0 ? vs0 + emax : 0x7fffffff;
+    uint32_t xmax = 0;
+#pragma unroll
+    for (int e = 0; e < PER; ++e)
+      if (e == emax) xmax = word_at(e);
+#pragma unroll
+    for (int o = 1; o < TPR; o <<= 1) {
       const float oy = __shfl_xor_sync(0xffffffffu, ymax, o);
       const int ov = __shfl_xor_sync(0xffffffffu, vmax, o);
+      const uint32_t ox = __shfl_xor_sync(0xffffffffu, xmax, o);
       if (oy > ymax || (oy == ymax && ov < vmax)) {
         ymax = oy;
         vmax = ov;
+        xmax = ox;
       }
     }
-    const uint32_t c3 = (uint32_t)(a.canvas_offset + bi) | (kStreamGumbel << 24);
     float best = -INFINITY;
     int barg = 0x7fffffff;
     if (draw && vmax != 0x7fffffff) {
-      // every lane evaluates the seed element's score identically
-      const Words4 w = philox((uint32_t)vmax >> 2, (uint32_t)l, (uint32_t)a.s, c3, a.key0, a.key1);
-      best = ymax + gumbel(pick_word(w, (uint32_t)vmax & 3u));
+      best = ymax + gumbel(xmax);
       barg = vmax;
       const float s0 = best;
-      uint32_t cur_call = 0xffffffffu;
-      Words4 cw{};
-      for (int e = 0; e < per; ++e) {
-        const int v = e0 + e;
+#pragma unroll
+      for (int e = 0; e < PER; ++e) {
+        const int v = vs0 + e;
         if (v >= a.V || v == vmax) continue;
-        if (((uint32_t)v >> 2) != cur_call) {
-          cur_call = (uint32_t)v >> 2;
-          cw = philox(cur_call, (uint32_t)l, (uint32_t)a.s, c3, a.key0, a.key1);
-        }
-        const uint32_t x = pick_word(cw, (uint32_t)v & 3u);
-        const float y = load_elem<DT>(rowp, v) * a.iT;
+        const uint32_t x = word_at(e);
+        const float y = zs[e] * a.iT;
         // can v beat the seed?  It needs g > s0 - y, i.e. -ln u < e^-(s0 - y);
         // -ln u >= 1 - u, so 1 - u >= e^-(s0 - y) (1e-4 relative margin) rules it out.
         const float tgap = s0 - y;
@@ -290,7 +360,8 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
         }
       }
     }
-    for (int o = 1; o < tpr; o <<= 1) {
+#pragma unroll
+    for (int o = 1; o < TPR; o <<= 1) {
       const float ob = __shfl_xor_sync(0xffffffffu, best, o);
       const int oa = __shfl_xor_sync(0xffffffffu, barg, o);
       if (ob > best || (ob == best && oa < barg)) {
@@ -308,7 +379,8 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
 // ---------------------------------------------------------------------------
 __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const float* sH,
                                 const int* sAm, const int* sSmp, const float* sPm,
-                                const uint8_t* sOpen, uint8_t* pick, unsigned long long* keys,
+                                const int* sPrev, const int* sTok, const uint8_t* sOpen,
+                                uint8_t* pick, unsigned long long* keys,
                                 unsigned long long* skeys) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int L = a.L;
@@ -321,9 +393,9 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
   for (int l = tid; l < L; l += kFinThreads) {
     pick[l] = 0;
     sumH += (double)sH[l];
-    if (a.s >= 1 && sAm[l] != a.prev_amax[row0 + l]) neq = 1;
+    if (a.s >= 1 && sAm[l] != sPrev[l]) neq = 1;
     if (!sOpen[l]) {
-      const int tok = a.canvas[row0 + l];
+      const int tok = sTok[l];
       if (tok < 0 || tok >= a.V) atomicOr(a.status, kStatusBadToken);
     } else if (!br) {
       ncand += (double)sH[l] <= a.gamma ? 1 : 0;
@@ -333,7 +405,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
   }
   const double totH = fin_block_sum(sumH, ctrl);
   const int any_neq = fin_block_sum_int(neq, ctrl);
-  const int stable_new = any_neq ? 0 : a.stable[bi] + 1;
+  const int stable_new = any_neq ? 0 : ctrl->stable_prev + 1;
   const double meanH = totH / (double)L;
   const bool fired = a.stop_enabled && stable_new >= a.stability_steps && meanH < a.tau;
   const bool last_step = a.s == a.N - 1;
@@ -440,65 +512,86 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
 
 // act_index[b]: index of canvas b among the canvases active at the start of
 // the step (-1 if it had stopped), written by the stream kernel.
-template <int DT>
-__global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThreads)
-    finish_kernel(const StepArgs a, const int32_t* act_index, const int32_t* n_act_ptr) {
-  griddep_wait();  // the stream kernel has completed and its writes are visible
-  extern __shared__ __align__(16) unsigned char smem[];
-  const FinLayout lay = fin_layout(a.L);
-  FinCtrl* ctrl = reinterpret_cast<FinCtrl*>(smem + lay.ctrl);
-  float* sH = reinterpret_cast<float*>(smem + lay.H);
-  int* sAm = reinterpret_cast<int*>(smem + lay.am);
-  int* sSmp = reinterpret_cast<int*>(smem + lay.smp);
-  float* sPm = reinterpret_cast<float*>(smem + lay.pm);
-  uint8_t* sOpen = smem + lay.open;
-  uint8_t* pick = smem + lay.pick;
-  unsigned long long* keys = reinterpret_cast<unsigned long long*>(smem + lay.keys);
-  unsigned long long* skeys = reinterpret_cast<unsigned long long*>(smem + lay.skeys);
-
-  cgr::cluster_group cluster = cgr::this_cluster();
-  const int rank = (int)cluster.block_rank();
-  const int bi = blockIdx.x / kFinCluster;
-  const int ai = act_index[bi];
-  if (ai < 0) return;  // uniform over the cluster: a stopped canvas is untouched
-  const int n_act = *n_act_ptr;
-  const unsigned long long NG =
-      (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
-
+template <int DT, int TPR>
+__device__ __forceinline__ void finish_rows(const StepArgs& a, const FinLayout& lay,
+                                            unsigned char* smem, cgr::cluster_group& cluster,
+                                            int bi, int ai, int rank, bool open,
+                                            unsigned long long NG) {
   const int rpc = fin_rows_per_cta(a.L);
-  const int tpr = fin_lanes_per_row(a.L);
   const int tid = threadIdx.x;
-  const int sub = tid / tpr, sl = tid % tpr;
+  const int sub = tid / TPR, sl = tid % TPR;
   const int l = rank * rpc + sub;
   const bool valid = sub < rpc && l < a.L;
-  const RowOut ro = DT == kBF16 ? finish_row<kBF16>(a, bi, ai, l, valid, tpr, sl, NG)
-                                : finish_row<kF32>(a, bi, ai, l, valid, tpr, sl, NG);
+  const RowOut ro = finish_row<DT, TPR>(a, bi, ai, l, valid, open, sl, NG);
   if (valid && sl == 0) {
     const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
     a.H_out[grow] = ro.H;
     a.amax_out[grow] = ro.amax;
     a.sample[grow] = ro.sample;
     a.pmax[grow] = ro.pmax;
-    sH[l] = ro.H;
-    sAm[l] = ro.amax;
-    sSmp[l] = ro.sample;
-    sPm[l] = ro.pmax;
-    sOpen[l] = a.committed[grow] == 0 ? 1 : 0;
+    // straight into cluster rank 0's shared memory
+    *cluster.map_shared_rank(reinterpret_cast<float*>(smem + lay.H) + l, 0) = ro.H;
+    *cluster.map_shared_rank(reinterpret_cast<int*>(smem + lay.am) + l, 0) = ro.amax;
+    *cluster.map_shared_rank(reinterpret_cast<int*>(smem + lay.smp) + l, 0) = ro.sample;
+    *cluster.map_shared_rank(reinterpret_cast<float*>(smem + lay.pm) + l, 0) = ro.pmax;
+    *cluster.map_shared_rank(smem + lay.open + l, 0) = open ? 1 : 0;
   }
-  cluster.sync();
-  if (rank == 0) {  // gather the other slices from the peers' shared memory
+}
+
+template <int DT>
+__global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThreads, 2)
+    finish_kernel(const StepArgs a, const int32_t* act_index, const int32_t* n_act_ptr) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const FinLayout lay = fin_layout(a.L);
+  FinCtrl* ctrl = reinterpret_cast<FinCtrl*>(smem + lay.ctrl);
+  cgr::cluster_group cluster = cgr::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int bi = blockIdx.x / kFinCluster;
+  const int tid = threadIdx.x;
+  const int rpc = fin_rows_per_cta(a.L);
+  const int tpr = fin_lanes_per_row(a.L);
+
+  // Before the stream kernel has finished: what the previous step left (the
+  // canvas state is written only by finish kernels, never by the stream
+  // kernel that runs now).
+  const int my_l = rank * rpc + tid / tpr;
+  const bool open = tid / tpr < rpc && my_l < a.L &&
+                    a.committed[(size_t)bi * (size_t)a.L + (size_t)my_l] == 0;
+  if (rank == 0) {
+    const size_t row0 = (size_t)bi * (size_t)a.L;
+    int* sPrev = reinterpret_cast<int*>(smem + lay.prev);
+    int* sTok = reinterpret_cast<int*>(smem + lay.tok);
     for (int i = tid; i < a.L; i += kFinThreads) {
-      const int owner = i / rpc;
-      if (owner == 0) continue;
-      sH[i] = *cluster.map_shared_rank(sH + i, owner);
-      sAm[i] = *cluster.map_shared_rank(sAm + i, owner);
-      sSmp[i] = *cluster.map_shared_rank(sSmp + i, owner);
-      sPm[i] = *cluster.map_shared_rank(sPm + i, owner);
-      sOpen[i] = *cluster.map_shared_rank(sOpen + i, owner);
+      sPrev[i] = a.prev_amax[row0 + i];
+      sTok[i] = a.canvas[row0 + i];
     }
+    if (tid == 0) ctrl->stable_prev = a.stable[bi];
   }
-  cluster.sync();  // peers stay resident until rank 0 has read them
-  if (rank == 0) canvas_epilogue(a, bi, ctrl, sH, sAm, sSmp, sPm, sOpen, pick, keys, skeys);
+  cluster.sync();  // every CTA of the cluster runs: its shared memory may be written
+
+  griddep_wait();  // the stream kernel has completed and its writes are visible
+  const int ai = act_index[bi];
+  if (ai < 0) return;  // uniform over the cluster: a stopped canvas is untouched
+  const int n_act = *n_act_ptr;
+  const unsigned long long NG =
+      (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
+  switch (tpr) {
+    case 2: finish_rows<DT, 2>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+    case 4: finish_rows<DT, 4>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+    case 8: finish_rows<DT, 8>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+    case 16: finish_rows<DT, 16>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+    default: finish_rows<DT, 32>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+  }
+  cluster.sync();  // rank 0 now holds every position's results
+  if (rank == 0)
+    canvas_epilogue(a, bi, ctrl, reinterpret_cast<const float*>(smem + lay.H),
+                    reinterpret_cast<const int*>(smem + lay.am),
+                    reinterpret_cast<const int*>(smem + lay.smp),
+                    reinterpret_cast<const float*>(smem + lay.pm),
+                    reinterpret_cast<const int*>(smem + lay.prev),
+                    reinterpret_cast<const int*>(smem + lay.tok), smem + lay.open,
+                    smem + lay.pick, reinterpret_cast<unsigned long long*>(smem + lay.keys),
+                    reinterpret_cast<unsigned long long*>(smem + lay.skeys));
 }
 
 // Initial canvas: uniform-random tokens (stream 2), nothing committed.

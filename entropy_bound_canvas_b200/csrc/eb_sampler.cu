@@ -2,7 +2,7 @@
 //
 // Validation, the device workspace, launch configuration and error codes.
 // A step is two kernels on the caller's stream: the persistent stream kernel
-// (eb_stream.cuh, sized to fill every SM) and the finish kernel
+// (eb_stream.cuh, one CTA per SM) and the finish kernel
 // (eb_finish.cuh, one 8-CTA cluster per canvas), launched as a programmatic
 // dependent of the first so that its launch overlaps the first one's end.
 // All the per-step arithmetic runs in those kernels.
@@ -37,8 +37,9 @@ struct eb_sampler {
   int device = 0;
   int sms = 0;
   int ng = 0;
-  int max_segs = 0;
-  KernelCfg k[2][2];  // stream kernel [dtype][tma]
+  int max_segs = 0;  // stream CTAs that can share one row
+  int nw = 0;        // records per (row, stream CTA)
+  KernelCfg k[2];     // stream kernel [dtype]
   KernelCfg fin[2];   // finish kernel [dtype]
   // workspace (one allocation)
   void* ws = nullptr;
@@ -92,26 +93,27 @@ int validate_config(const eb_config_t* c) {
   return EB_OK;
 }
 
-template <int DT, bool TMA>
+template <int DT>
 int setup_kernel(eb_sampler* h, const cudaDeviceProp& prop) {
-  KernelCfg& kc = h->k[DT][TMA ? 1 : 0];
+  KernelCfg& kc = h->k[DT];
   const ebk::StreamLayout lay = ebk::stream_layout<DT>(h->cfg.B);
-  kc.fn = reinterpret_cast<const void*>(&ebk::stream_kernel<DT, TMA>);
+  kc.fn = reinterpret_cast<const void*>(&ebk::stream_kernel<DT>);
   kc.smem = lay.total;
   if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
-  if (cudaFuncSetAttribute(ebk::stream_kernel<DT, TMA>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kc.smem) != cudaSuccess)
+  if (cudaFuncSetAttribute(ebk::stream_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kc.smem) != cudaSuccess)
     return EB_ERR_CUDA;
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::stream_kernel<DT, TMA>,
-                                                    ebk::StreamShape<DT>::kThreads, kc.smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::stream_kernel<DT>,
+                                                    ebk::StreamShape<DT>::kThreads, kc.smem) !=
+          cudaSuccess ||
       per_sm < 1)
     return EB_ERR_CUDA;
+  // one persistent CTA per SM, fewer if there are fewer stage-sized tiles
   const uint64_t groups = (uint64_t)h->cfg.B * (uint64_t)h->cfg.L * (uint64_t)h->ng;
-  const uint64_t want =
-      (groups + ebk::StreamShape<DT>::kTileGroups - 1) / ebk::StreamShape<DT>::kTileGroups;
-  kc.grid = (int)std::min<uint64_t>((uint64_t)per_sm * (uint64_t)prop.multiProcessorCount,
-                                    std::max<uint64_t>(1, want));
+  const uint64_t want = (groups + ebk::StreamShape<DT>::kStageGroups - 1) /
+                        ebk::StreamShape<DT>::kStageGroups;
+  kc.grid = (int)std::min<uint64_t>((uint64_t)prop.multiProcessorCount, std::max<uint64_t>(1, want));
   return EB_OK;
 }
 
@@ -173,10 +175,8 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   h->sms = prop.multiProcessorCount;
   h->ng = (int)(((int64_t)cfg->V + ebk::kGroup - 1) / ebk::kGroup);
 
-  if ((rc = setup_kernel<ebk::kF32, true>(h, prop)) != EB_OK ||
-      (rc = setup_kernel<ebk::kF32, false>(h, prop)) != EB_OK ||
-      (rc = setup_kernel<ebk::kBF16, true>(h, prop)) != EB_OK ||
-      (rc = setup_kernel<ebk::kBF16, false>(h, prop)) != EB_OK ||
+  if ((rc = setup_kernel<ebk::kF32>(h, prop)) != EB_OK ||
+      (rc = setup_kernel<ebk::kBF16>(h, prop)) != EB_OK ||
       (rc = setup_finish<ebk::kF32>(h, prop)) != EB_OK ||
       (rc = setup_finish<ebk::kBF16>(h, prop)) != EB_OK) {
     delete h;
@@ -186,16 +186,16 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   // least floor(L ng / G) groups, so a row meets at most
   // floor((ng - 1) G / (L ng)) + 2 of them.
   int gmax = 0;
-  for (int d = 0; d < 2; ++d)
-    for (int t = 0; t < 2; ++t) gmax = std::max(gmax, h->k[d][t].grid);
+  for (int d = 0; d < 2; ++d) gmax = std::max(gmax, h->k[d].grid);
   const uint64_t Lng = (uint64_t)cfg->L * (uint64_t)h->ng;
   const uint64_t segs = ((uint64_t)(h->ng - 1) * (uint64_t)gmax) / Lng + 2;
   h->max_segs = (int)std::min<uint64_t>((uint64_t)gmax, segs);
+  h->nw = ebk::stream_consumer_warps();
 
   const size_t BL = (size_t)cfg->B * (size_t)cfg->L;
   size_t off = 0;
   const size_t o_part = off;
-  off = align256(off + sizeof(Partial) * BL * (size_t)h->max_segs);
+  off = align256(off + sizeof(Partial) * BL * (size_t)h->max_segs * (size_t)h->nw);
   const size_t o_status = off;
   off = align256(off + sizeof(uint32_t));
   const size_t o_act = off;
@@ -252,6 +252,7 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   if (!h || !logits || !canvas || !committed || !entropies || !argmax || !stop_flags)
     return EB_ERR_INVALID_ARG;
   if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
+  if ((uintptr_t)logits % (dtype == EB_F32 ? 4u : 2u) != 0) return EB_ERR_INVALID_ARG;
   const eb_config_t& c = h->cfg;
   if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
   if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
@@ -286,6 +287,7 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.s = step;
   a.N = c.num_steps;
   a.max_segs = h->max_segs;
+  a.nw = h->nw;
   a.rule = c.rule;
   a.quota = c.quota;
   a.stability_steps = c.stability_steps;
@@ -301,10 +303,10 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.key1 = (uint32_t)(c.seed >> 32);
 
   const size_t elt = dtype == EB_F32 ? 4 : 2;
-  const bool tma = ((uintptr_t)logits % 16 == 0) && (((size_t)c.V * elt) % 16 == 0);
-  const KernelCfg& kc = h->k[dtype][tma ? 1 : 0];
+  const bool vec = ((uintptr_t)logits % 16 == 0) && (((size_t)c.V * elt) % 16 == 0);
+  const KernelCfg& kc = h->k[dtype];
   a.G1 = kc.grid;
-  a.vec_ok = tma ? 1 : 0;
+  a.vec_ok = vec ? 1 : 0;
   void* args[] = {&a};
   if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), args, kc.smem, st) !=
       cudaSuccess)

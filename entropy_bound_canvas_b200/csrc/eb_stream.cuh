@@ -1,91 +1,109 @@
 // eb_stream.cuh -- first kernel of a sampler step: one pass over every logit
 // of every active canvas.
 //
-// The active rows' 64-logit groups are numbered g = row * ng + j; stream CTA
-// c of G owns the contiguous range [c NG / G, (c + 1) NG / G), so every CTA
-// reads the same number of bytes (to within one group).  A range is walked in
-// tiles of up to kTileGroups groups that never straddle a row.  Lane 0 of the
-// last warp copies tiles into a kStages-deep shared-memory ring with 1-D bulk
-// copies (the TMA engine, no multicast, L2 evict-first); the other warps (the
-// "consumer" threads) reduce one group each per tile: the group maximum,
-// sum 2^d, sum 2^d d and, for open positions, a Gumbel-perturbed group
-// log-partition.  At the end of each row segment the consumer partials are
-// merged and written as one Partial record; nothing else crosses CTAs, and no
-// CTA waits for another.
+// Work split.  The active rows' 64-logit groups are numbered g = row ng + j
+// (row = active canvas index * L + position).  Stream CTA c of G (one per SM)
+// owns the contiguous range [c NG / G, (c + 1) NG / G): every CTA reads the
+// same number of bytes to within one group, and a row meets only a few CTAs.
+//
+// Inside a CTA.  The producer warp walks the range in tiles of up to
+// kStageGroups groups that never straddle a row.  For each tile it writes the
+// tile's description and, for an open position, the group-stream Philox
+// words of the tile's groups into the stage's header in shared memory; lane 0
+// then copies the tile into a kStages-deep ring with one 1-D bulk copy (the
+// TMA engine, no multicast, L2 evict-first).  A tile is cut into sub-tiles of
+// 64 groups, dealt round-robin to the consumer warps (a fixed assignment, so
+// every run sums in the same order).  A lane reduces two groups of its warp's
+// sub-tile; the warp shares one running maximum per row (WarpAcc), so its
+// lanes' sums stay relative to the same reference and the Gumbel race runs
+// against the warp's best.  When a warp moves on to another row it sums its
+// lanes and writes one Partial record for (row, CTA, warp); it writes an
+// empty record for
+// each row of its CTA's range that it never touched, so the finish kernel
+// only ever reads records written during this step.
 #pragma once
 
 #include "eb_common.cuh"
 
 namespace ebk {
 
-#ifndef EB_STREAM_WARPS_BF16
-#define EB_STREAM_WARPS_BF16 4
+#ifndef EB_STREAM_CONSUMER_WARPS
+#define EB_STREAM_CONSUMER_WARPS 12
 #endif
-#ifndef EB_STREAM_WARPS_F32
-#define EB_STREAM_WARPS_F32 4
+#ifndef EB_STREAM_STAGES
+#define EB_STREAM_STAGES 6
 #endif
-#ifndef EB_STREAM_CTAS_BF16
-#define EB_STREAM_CTAS_BF16 4
-#endif
-#ifndef EB_STREAM_CTAS_F32
-#define EB_STREAM_CTAS_F32 2
+#ifndef EB_STREAM_STAGE_KB
+#define EB_STREAM_STAGE_KB 32
 #endif
 
-constexpr int kStages = 3;
+constexpr int kStages = EB_STREAM_STAGES;
 
-// Shape of a stream CTA per logits dtype: consumer warps (one 64-logit group
-// per consumer thread per tile), tile size, threads (consumers + 1 producer
-// warp) and the CTAs meant to share an SM.  bf16: 4 consumer warps, 16 KB
-// tiles, a 48 KB ring, 4 CTAs per SM.  Measured on the 1 x 256 x 262144 bf16
-// canvas this beat one 16-warp CTA per SM (64 KB tiles) by 11 %: four
-// independent rings keep more bulk copies in flight per SM, and a CTA that
-// falls behind holds back only its own quarter of the SM.  fp32: 4 consumer
-// warps, 32 KB tiles, 2 CTAs per SM (the fp32 consumer needs ~160 registers).
+// Shape of the stream CTA: kConsumerWarps consumer warps + 1 producer warp,
+// a ring of kStages stages of kStageBytes each (192 KB with the defaults:
+// one CTA per SM).  Twelve consumer warps, each lane reducing two groups at
+// a time, keep the SM's MUFU and FMA pipes busy.
 template <int DT>
 struct StreamShape {
-  static constexpr int kWarps = DT == kBF16 ? EB_STREAM_WARPS_BF16 : EB_STREAM_WARPS_F32;
-  static constexpr int kCtasPerSM = DT == kBF16 ? EB_STREAM_CTAS_BF16 : EB_STREAM_CTAS_F32;
-  static constexpr int kConsumers = kWarps * 32;
-  static constexpr int kThreads = kConsumers + 32;
-  static constexpr int kTileGroups = kConsumers;
-  static constexpr int kTileBytes = kTileGroups * kGroup * elt_bytes(DT);
+  static constexpr int kConsumerWarps = EB_STREAM_CONSUMER_WARPS;
+  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kStageBytes = EB_STREAM_STAGE_KB * 1024;
+  // room for a copy widened to 16-byte boundaries; 128-byte aligned stages
+  static constexpr int kStageStride = kStageBytes + 128;
+  static constexpr int kStageGroups = kStageBytes / (kGroup * elt_bytes(DT));
+  static constexpr int kSubGroups = 64;  // groups per sub-tile: two per lane
+  static constexpr int kSubPerStage = kStageGroups / kSubGroups;
+  static_assert(kSubPerStage >= 1 && (kSubPerStage & (kSubPerStage - 1)) == 0,
+                "sub-tiles per stage must be a power of two");
 };
 
 __host__ __device__ constexpr int stream_threads(int dt) {
   return dt == kBF16 ? StreamShape<kBF16>::kThreads : StreamShape<kF32>::kThreads;
 }
-__host__ __device__ constexpr int stream_tile_groups(int dt) {
-  return dt == kBF16 ? StreamShape<kBF16>::kTileGroups : StreamShape<kF32>::kTileGroups;
-}
+__host__ __device__ constexpr int stream_consumer_warps() { return EB_STREAM_CONSUMER_WARPS; }
 
 struct StreamCtrl {
-  int n_act;
   int abort;
-  int issued;
-  int pad;
+  int issued;  // tiles whose bulk copy has been issued
+  int n_sub;   // sub-tiles of this CTA's range
   int wcnt[32];
 };
 
+// What the producer tells the consumers about the tile in a stage.
+struct TileMeta {
+  int r;         // active row index
+  int j0;        // first group of the tile within the row
+  int cnt;       // groups in the tile
+  int bi;        // canvas
+  int l;         // position
+  int sampling;  // open position of a sampled (not greedy) run
+  int delta;     // byte offset of the tile's first logit in the stage
+  int pad;
+};
+
 struct StreamLayout {
-  uint32_t bars, ctrl, red, act, ring, total;
+  uint32_t bars, ctrl, meta, words, act, ring, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 template <int DT>
 __host__ __device__ inline StreamLayout stream_layout(int B) {
+  using Sh = StreamShape<DT>;
   StreamLayout y;
   uint32_t o = 0;
   y.bars = o;
   o = align_up(o + 16u * kStages, 16);
   y.ctrl = o;
   o = align_up(o + (uint32_t)sizeof(StreamCtrl), 16);
-  y.red = o;
-  o = align_up(o + (uint32_t)sizeof(Partial) * StreamShape<DT>::kWarps, 16);
+  y.meta = o;
+  o = align_up(o + (uint32_t)sizeof(TileMeta) * kStages, 16);
+  y.words = o;
+  o = align_up(o + 4u * (uint32_t)Sh::kStageGroups * kStages, 16);
   y.act = o;
   o = align_up(o + 2u * (uint32_t)B, 128);
   y.ring = o;
-  o += (uint32_t)kStages * (uint32_t)StreamShape<DT>::kTileBytes;
+  o += (uint32_t)kStages * (uint32_t)Sh::kStageStride;
   y.total = o;
   return y;
 }
@@ -98,8 +116,9 @@ struct Tile {
   int l;        // position of the row
 };
 
-// Walks a CTA's group range in tiles of up to tg groups; divides only once,
-// at the start.
+// Walks a CTA's group range in tiles that end at the row's multiples of tg
+// groups (so a tile after the first of a row segment starts on a Philox
+// call boundary); divides only once, at the start.
 struct TileIter {
   unsigned long long g, g_hi;
   int ng, L, tg;
@@ -116,7 +135,8 @@ struct TileIter {
   __device__ __forceinline__ bool next(Tile& t) {
     if (g >= g_hi) return false;
     int cnt = ng - j0;
-    if (cnt > tg) cnt = tg;
+    const int to_edge = tg - j0 % tg;  // tiles end on multiples of tg within a row
+    if (cnt > to_edge) cnt = to_edge;
     if ((unsigned long long)cnt > g_hi - g) cnt = (int)(g_hi - g);
     t.r = r;
     t.j0 = j0;
@@ -136,6 +156,22 @@ struct TileIter {
     return true;
   }
 };
+
+// Tiles of the range [lo, hi), the same cut as TileIter: a row segment
+// covering groups [a, b) of its row has ceil(b / tg) - floor(a / tg) tiles.
+__device__ __forceinline__ int count_tiles(unsigned long long lo, unsigned long long hi, int ng,
+                                           int tg) {
+  int n = 0;
+  while (lo < hi) {
+    const unsigned long long r = lo / (unsigned long long)ng;
+    unsigned long long e = (r + 1ull) * (unsigned long long)ng;
+    if (e > hi) e = hi;
+    const int a = (int)(lo - r * (unsigned long long)ng), b = (int)(e - r * (unsigned long long)ng);
+    n += (b + tg - 1) / tg - a / tg;
+    lo = e;
+  }
+  return n;
+}
 
 // Active canvases in index order, from the stop flags as they were when the
 // step began (only the finish kernel, after this one, writes them).
@@ -159,217 +195,274 @@ __device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int 
   return base;
 }
 
-// End of a row segment: merge the 128 thread partials and write the CTA's
-// partial for the row into its slot (CTA index minus the row's first CTA).
-template <int DT>
-__device__ __forceinline__ void flush_segment(const StepArgs& a, Partial& acc, long long r, int bi,
-                                              int l, unsigned long long NG, Partial* red, int tid) {
-  using Sh = StreamShape<DT>;
-  const int lane = tid & 31, warp = tid >> 5;
-  warp_merge(acc, a.c2);
-  if (lane == 0) red[warp] = acc;
-  consumer_sync(Sh::kConsumers);
-  if (tid == 0) {
-    Partial P = red[0];
-    for (int w = 1; w < Sh::kWarps; ++w) merge(P, red[w], a.c2);
-    const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
-    const int slot =
-        (int)blockIdx.x - cta_of((unsigned long long)r * (unsigned long long)a.ng, NG, gridDim.x);
-    a.partials[grow * (size_t)a.max_segs + (size_t)slot] = P;
-  }
-  consumer_sync(Sh::kConsumers);
-}
+#ifndef EB_STREAM_MAXNREG
+#define EB_STREAM_MAXNREG 128
+#endif
 
-template <int DT, bool TMA>
-__global__ void __launch_bounds__(StreamShape<DT>::kThreads, StreamShape<DT>::kCtasPerSM)
-    stream_kernel(const StepArgs a) {
+// 128 registers keep the two-group consumer loop free of spills; with 12
+// consumer warps the CTA then holds 53 K of the SM's 64 K registers.
+template <int DT>
+__global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
   using Sh = StreamShape<DT>;
+  using IO = GroupIO<DT>;
   extern __shared__ __align__(128) unsigned char smem[];
   const StreamLayout lay = stream_layout<DT>(a.B);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
   uint64_t* empty = full + kStages;
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(smem + lay.ctrl);
-  Partial* red = reinterpret_cast<Partial*>(smem + lay.red);
+  TileMeta* meta = reinterpret_cast<TileMeta*>(smem + lay.meta);
+  uint32_t* words = reinterpret_cast<uint32_t*>(smem + lay.words);
   uint16_t* act = reinterpret_cast<uint16_t*>(smem + lay.act);
   unsigned char* ring = smem + lay.ring;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   if (tid == 0) {
     for (int st = 0; st < kStages; ++st) {
-      mbar_init(&full[st], 1);
-      mbar_init(&empty[st], Sh::kWarps);
+      mbar_init(&full[st], 2);  // the copy's arrival (+ bytes) and the header's
+      mbar_init(&empty[st], Sh::kSubPerStage);
     }
     ctrl->abort = 0;
     ctrl->issued = 0;
     fence_mbar_init();
   }
-  const int n = build_active_list(a.stop_flags, a.B, act, ctrl->wcnt, Sh::kThreads);
-  if (tid == 0) ctrl->n_act = n;
+  const int n_act = build_active_list(a.stop_flags, a.B, act, ctrl->wcnt, Sh::kThreads);
   if (blockIdx.x == 0) {  // publish the active list for the finish kernel
     for (int b = tid; b < a.B; b += Sh::kThreads) a.act_index[b] = -1;
     __syncthreads();
-    for (int i = tid; i < n; i += Sh::kThreads) a.act_index[act[i]] = i;
-    if (tid == 0) *a.n_act = n;
+    for (int i = tid; i < n_act; i += Sh::kThreads) a.act_index[act[i]] = i;
+    if (tid == 0) *a.n_act = n_act;
   }
-  __syncthreads();
-
-  const int n_act = ctrl->n_act;
   const int G = gridDim.x;
   const unsigned long long NG =
       (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
   const unsigned long long g_lo = range_start(blockIdx.x, NG, G);
   const unsigned long long g_hi = range_start(blockIdx.x + 1, NG, G);
+  if (tid == 0) ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
+  __syncthreads();
+  // The finish kernel may be scheduled from now on, wherever an SM has room:
+  // its CTAs load what the previous step left and then wait for this grid's
+  // completion (griddepcontrol.wait) before reading anything it writes.
+  griddep_launch_dependents();
+
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
   const char* logits = reinterpret_cast<const char*>(a.logits);
 
-  if (warp == Sh::kWarps) {
+  if (warp == Sh::kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (TMA && lane == 0) {
-      const uint64_t policy = evict_first_policy();
-      TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kTileGroups);
-      Tile t;
-      int k = 0;
-      while (it.next(t)) {
-        const int st = k % kStages;
-        if (k >= kStages) {
-          if (!mbar_wait(&empty[st], (uint32_t)((k / kStages) - 1) & 1u)) {
+    const uint64_t policy = evict_first_policy();
+    TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kStageGroups);
+    Tile t;
+    int k = 0, st = 0;
+    uint32_t ph = 0;  // parity of the current pass over the ring
+    long long row_seen = -1;
+    int bi = 0, samp = 0;
+    while (it.next(t)) {
+      if (k >= kStages) {
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait(&empty[st], ph ^ 1u) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
             atomicOr(a.status, kStatusTimeout);
             *(volatile int*)&ctrl->abort = 1;
           }
+          break;
         }
-        if (*(volatile int*)&ctrl->abort) break;
-        const size_t grow = (size_t)act[t.ai] * (size_t)a.L + (size_t)t.l;
-        const size_t e0 = (size_t)t.j0 * kGroup;
-        size_t nel = (size_t)t.cnt * kGroup;
-        if (e0 + nel > (size_t)a.V) nel = (size_t)a.V - e0;
-        const uint32_t bytes = (uint32_t)(nel * elt_bytes(DT));
-        mbar_arrive_expect_tx(&full[st], bytes);
-        bulk_load(ring + (size_t)st * Sh::kTileBytes, logits + grow * row_bytes + e0 * elt_bytes(DT),
-                  bytes, &full[st], policy);
-        ++k;
-        *(volatile int*)&ctrl->issued = k;
+      }
+      if (*(volatile int*)&ctrl->abort) break;
+      if (t.r != row_seen) {
+        row_seen = t.r;
+        bi = act[t.ai];
+        samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
+      }
+      const char* src = logits + ((size_t)bi * (size_t)a.L + (size_t)t.l) * row_bytes +
+                        (size_t)t.j0 * kGroup * elt_bytes(DT);
+      size_t nel = (size_t)t.cnt * kGroup;
+      if ((size_t)t.j0 * kGroup + nel > (size_t)a.V) nel = (size_t)a.V - (size_t)t.j0 * kGroup;
+      // The copy is widened to 16-byte boundaries: at most 15 bytes on each
+      // side, inside the 16-byte blocks that hold the tile's first and last
+      // logits.
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~(uintptr_t)15;
+      const uintptr_t a1 =
+          (reinterpret_cast<uintptr_t>(src) + nel * elt_bytes(DT) + 15) & ~(uintptr_t)15;
+      if (lane == 0) {
+        TileMeta m;
+        m.r = (int)t.r;
+        m.j0 = t.j0;
+        m.cnt = t.cnt;
+        m.bi = bi;
+        m.l = t.l;
+        m.sampling = samp;
+        m.delta = (int)(reinterpret_cast<uintptr_t>(src) - a0);
+        m.pad = 0;
+        meta[st] = m;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(a1 - a0));
+        bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
+                  (uint32_t)(a1 - a0), &full[st], policy);
+      }
+      if (samp) {  // while the copy is in flight: the tile's group-stream words
+        uint32_t* wd = words + st * Sh::kStageGroups;
+        const int c0 = t.j0 >> 2, c1 = (t.j0 + t.cnt - 1) >> 2;
+        const uint32_t c3 = (uint32_t)(a.canvas_offset + bi) | (kStreamGroup << 24);
+        for (int c = c0 + lane; c <= c1; c += 32) {
+          const Words4 w = philox((uint32_t)c, (uint32_t)t.l, (uint32_t)a.s, c3, a.key0, a.key1);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int j = 4 * c + q - t.j0;
+            if (j >= 0 && j < t.cnt) wd[j] = w.w[q];
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&full[st]);  // header (meta, words) complete
+        st_release_shared(&ctrl->issued, k + 1);
+      }
+      ++k;
+      if (++st == kStages) {
+        st = 0;
+        ph ^= 1u;
       }
     }
   } else {
     // ------------------------------------------------------------ consumers
-    TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kTileGroups);
-    Tile t;
-    int k = 0;
+    const int n_sub = ctrl->n_sub;
+    const long long r_first = (long long)(g_lo / (unsigned long long)a.ng);
+    const long long r_end =
+        g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
+    // slot of this CTA among the CTAs of its first row; later rows start in it
+    const int seg_first =
+        (int)blockIdx.x - cta_of((unsigned long long)r_first * (unsigned long long)a.ng, NG, G);
+    const size_t spr = (size_t)(a.max_segs * a.nw);
+    auto record_of = [&](long long r, int bi, int l) {
+      const int seg = r == r_first ? seg_first : 0;
+      return ((size_t)bi * (size_t)a.L + (size_t)l) * spr + (size_t)(seg * a.nw + warp);
+    };
     long long cur_r = -1;
-    int bi = 0, l = 0;
-    bool sampling = false;
-    Partial acc = empty_partial();
-    // Per-warp cache of group-stream Philox words for three tiles of a row.
-    Words4 wc{};
-    bool wc_valid = false;
-    int wc_jw0 = 0;
-    const int rot = tid;  // piece rotation for bank-conflict-free reads
+    long long next_r = r_first;  // first row of the range this warp still owes a record
+    size_t cur_rec = 0;
+    int sampling = 0;
+    WarpAcc A;
+    warp_reset(A);
+    const int rot = lane;
 
-    while (it.next(t)) {
-      if (t.r != cur_r) {
-        if (cur_r >= 0) flush_segment<DT>(a, acc, cur_r, bi, l, NG, red, tid);
-        cur_r = t.r;
-        acc = empty_partial();
-        wc_valid = false;
-        bi = act[t.ai];
-        l = t.l;
-        sampling = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)l] == 0;
+    auto owe_empty = [&](long long upto) {
+      for (; next_r < upto; ++next_r) {
+        if (lane == 0) {
+          const int ai = (int)(next_r / a.L);
+          const int l = (int)(next_r - (long long)ai * a.L);
+          a.partials[record_of(next_r, act[ai], l)] = empty_partial();
+        }
       }
+    };
+    auto flush = [&]() {
+      const Partial P = warp_record(A, a.iT);
+      if (lane == 0) a.partials[cur_rec] = P;
+    };
+
+    // Sub-tiles are dealt round-robin: warp w takes w, w + nw, w + 2 nw, ...
+    for (int u = warp; u < n_sub; u += Sh::kConsumerWarps) {
+      if (*(volatile int*)&ctrl->abort) break;
+      const int k = u / Sh::kSubPerStage;
+      const int sub = u & (Sh::kSubPerStage - 1);
       const int st = k % kStages;
-      const int j = t.j0 + tid;
-      float lse = -INFINITY;
-      if (TMA) {
-        bool ok = true;
-        if (!*(volatile int*)&ctrl->abort) ok = mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u);
-        if (!ok) {
+      // A warp may run up to a few sub-tiles ahead of the ring, past the
+      // stage's current phase; the parity of the full barrier is only
+      // unambiguous once the producer has issued tile k (which it does after
+      // the stage's previous tile, k - kStages, was released).
+      if (!wait_counter_above(&ctrl->issued, k) ||
+          !mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u)) {
+        if (lane == 0) {
           atomicOr(a.status, kStatusTimeout);
           *(volatile int*)&ctrl->abort = 1;
         }
+        break;
       }
-      if (tid < t.cnt) {
-        const int glen = (a.V - j * kGroup) < kGroup ? (a.V - j * kGroup) : kGroup;
-        GroupStat gs;
-        if (TMA) {
-          const unsigned char* gp =
-              ring + (size_t)st * Sh::kTileBytes + (size_t)tid * kGroup * elt_bytes(DT);
-          if (glen == kGroup) {
-            gs = DT == kBF16 ? group_bf16_full(gp, rot, a.c2) : group_f32_full(gp, rot, a.c2);
-          } else {
-            gs = group_scalar<DT>(gp, glen, a.c2);
+      const TileMeta m = meta[st];
+      if (m.r != cur_r) {
+        if (cur_r >= 0) flush();
+        owe_empty(m.r);
+        cur_r = m.r;
+        next_r = cur_r + 1;
+        cur_rec = record_of(cur_r, m.bi, m.l);
+        sampling = m.sampling;
+        warp_reset(A);
+      }
+      const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
+      if (sub * Sh::kSubGroups < m.cnt) {  // warp-uniform
+        const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
+        const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
+        const unsigned char* gp0 = sbase + (size_t)(has0 ? gl0 : 0) * kGroup * elt_bytes(DT);
+        const unsigned char* gp1 = has1 ? sbase + (size_t)gl1 * kGroup * elt_bytes(DT) : gp0;
+        const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
+        const int len0 = has0 ? min(kGroup, a.V - j0 * kGroup) : 0;
+        const int len1 = has1 ? min(kGroup, a.V - j1 * kGroup) : 0;
+        const bool fast = a.vec_ok && (!has0 || len0 == kGroup) && (!has1 || len1 == kGroup);
+        float mg0, mg1;
+        if (fast) {
+          mg0 = IO::max_of(gp0, rot);
+          mg1 = IO::max_of(gp1, rot);
+        } else {
+          mg0 = has0 ? group_max_safe<DT>(gp0, len0) : -INFINITY;
+          mg1 = has1 ? group_max_safe<DT>(gp1, len1) : -INFINITY;
+        }
+        if (!has0) mg0 = -INFINITY;
+        if (!has1) mg1 = -INFINITY;
+        warp_raise(A, fmaxf(mg0, mg1), mg0 >= mg1 ? j0 : j1, a.c2);
+        float S0 = 0.f, W0 = 0.f, S1 = 0.f, W1 = 0.f;
+        if (fast) {
+          IO::exp2_of(gp0, gp1, rot, a.c2, A.M, A.M, S0, W0, S1, W1);
+          // -inf (or other non-finite) logits: redo the group term by term
+          if (!(W0 >= -3.0e38f)) {
+            const float2 q = group_sums_safe<DT>(gp0, kGroup, a.c2, A.M);
+            S0 = q.x;
+            W0 = q.y;
+          }
+          if (!(W1 >= -3.0e38f)) {
+            const float2 q = group_sums_safe<DT>(gp1, kGroup, a.c2, A.M);
+            S1 = q.x;
+            W1 = q.y;
           }
         } else {
-          const char* gp = logits + ((size_t)bi * (size_t)a.L + (size_t)l) * row_bytes +
-                           (size_t)j * kGroup * elt_bytes(DT);
-          gs = group_scalar<DT>(gp, glen, a.c2);
-        }
-        fold_group(acc, gs, j, a.c2);
-        // group log-partition in natural units: ln2 (m c2 + log2 S)
-        if (sampling) lse = 0.6931471805599453f * fmaf(gs.m, a.c2, lg2(gs.S));
-      }
-      if (TMA) {
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
-      }
-      if (sampling) {
-        // Group-level Gumbel.  The 32 groups of this warp in one tile need at
-        // most 9 Philox calls (4 words each); lanes 0-26 compute the calls of
-        // this and the next two tiles of the row segment at once (the warp's
-        // groups advance by one tile, 128 groups, per tile) and every lane
-        // picks its word by shuffle.
-        const bool need = tid < t.cnt && lse + kGumbelMax >= acc.gscore;
-        if (__ballot_sync(0xffffffffu, need)) {
-          const int jw = t.j0 + warp * 32;
-          int dj = jw - wc_jw0;
-          if (!wc_valid || dj < 0 || dj >= 3 * Sh::kTileGroups || (dj % Sh::kTileGroups) != 0) {
-            wc_valid = true;
-            wc_jw0 = jw;
-            dj = 0;
-            if (lane < 27)
-              wc = philox((uint32_t)(jw >> 2) + 32u * (uint32_t)(lane / 9) + (uint32_t)(lane % 9),
-                          (uint32_t)l, (uint32_t)a.s,
-                          (uint32_t)(a.canvas_offset + bi) | (kStreamGroup << 24), a.key0, a.key1);
+          if (has0) {
+            const float2 q = group_sums_safe<DT>(gp0, len0, a.c2, A.M);
+            S0 = q.x;
+            W0 = q.y;
           }
-          const int src = 9 * (dj / Sh::kTileGroups) + (((jw & 3) + lane) >> 2);
-          const uint32_t x0 = __shfl_sync(0xffffffffu, wc.w[0], src);
-          const uint32_t x1 = __shfl_sync(0xffffffffu, wc.w[1], src);
-          const uint32_t x2 = __shfl_sync(0xffffffffu, wc.w[2], src);
-          const uint32_t x3 = __shfl_sync(0xffffffffu, wc.w[3], src);
-          if (need) {
-            const uint32_t sel = (uint32_t)j & 3u;
-            const uint32_t x = sel == 0 ? x0 : sel == 1 ? x1 : sel == 2 ? x2 : x3;
-            // This group wins only if g > t = best - lse, i.e. E = -ln u <
-            // e^-t.  Since E >= 1 - u, a group with 1 - u >= e^-t (checked
-            // with a 1e-4 relative margin) cannot win: skip its logarithms.
-            const float tgap = acc.gscore - lse;
-            bool cand = true;
-            if (tgap > -2.0f) cand = one_minus_u(x) < ex2(-1.4426950408889634f * tgap) * 1.0001f;
-            if (cand) {
-              const float sc = lse + gumbel(x);
-              if (sc > acc.gscore) {
-                acc.gscore = sc;
-                acc.gidx = j;
-              }
-            }
+          if (has1) {
+            const float2 q = group_sums_safe<DT>(gp1, len1, a.c2, A.M);
+            S1 = q.x;
+            W1 = q.y;
           }
         }
+        if (has0) warp_fold(A, S0, W0, j0);
+        if (has1) warp_fold(A, S1, W1, j1);
+        if (sampling) {
+          const uint32_t* wd = words + st * Sh::kStageGroups;
+          float Rl = A.R;
+          int gbl = 0x7fffffff;
+          if (has0) lane_race(Rl, gbl, S0, wd[gl0], j0);
+          if (has1) lane_race(Rl, gbl, S1, wd[gl1], j1);
+          warp_race_merge(A, Rl, gbl);
+        }
       }
-      ++k;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
     }
-    if (cur_r >= 0) flush_segment<DT>(a, acc, cur_r, bi, l, NG, red, tid);
+    if (cur_r >= 0) flush();
+    owe_empty(r_end);
+  }
 
-    // After an abort, wait (bounded) for bulk copies still in flight into
-    // this CTA's shared memory before it may exit.
-    if (TMA && tid == 0 && *(volatile int*)&ctrl->abort) {
-      const int issued = *(volatile int*)&ctrl->issued;
-      for (int st = 0; st < kStages && st < issued; ++st) {
-        const int n2 = (issued - st + kStages - 1) / kStages;
-        mbar_wait(&full[st], (uint32_t)(n2 - 1) & 1u);
-      }
+  __syncthreads();
+  // After an abort, wait (bounded) for bulk copies still in flight into this
+  // CTA's shared memory before it may exit.
+  if (tid == 0 && *(volatile int*)&ctrl->abort) {
+    const int issued = ld_acquire_shared(&ctrl->issued);
+    for (int st = 0; st < kStages && st < issued; ++st) {
+      const int n2 = (issued - st + kStages - 1) / kStages;
+      mbar_wait(&full[st], (uint32_t)(n2 - 1) & 1u);
     }
   }
-  // Let the finish kernel's CTAs be scheduled; it still waits for this
-  // grid's completion (and memory) before reading anything.
-  griddep_launch_dependents();
 }
 
 }  // namespace ebk
