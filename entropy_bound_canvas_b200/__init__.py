@@ -83,6 +83,8 @@ def _lib():
         L.eb_sampler_draws.restype = i32
         L.eb_sampler_set_state.argtypes = [vp, vp, vp, i32, vp]
         L.eb_sampler_set_state.restype = i32
+        L.eb_sampler_set_split_event.argtypes = [vp, vp]
+        L.eb_sampler_set_split_event.restype = i32
         L.eb_sampler_workspace_bytes.argtypes = [vp]
         L.eb_sampler_workspace_bytes.restype = C.c_size_t
         L.eb_sampler_destroy.argtypes = [vp]
@@ -251,6 +253,16 @@ class EBSampler:
         _check(_lib().eb_sampler_set_state(
             self._h, self._ptr(prev_argmax, torch.int32, (self.B, self.L), "prev_argmax"),
             sp, next_step, self._stream()), "eb_sampler_set_state")
+
+    def set_split_event(self, event=None):
+        """Record `event` (a torch.cuda.Event, or None to stop) between the two
+        kernels of every following step, for timing them apart."""
+        ptr = None
+        if event is not None:
+            if not event.cuda_event:  # torch creates the CUDA event on first record
+                event.record(_torch().cuda.current_stream(self.device))
+            ptr = C.c_void_p(event.cuda_event)
+        _check(_lib().eb_sampler_set_split_event(self._h, ptr), "eb_sampler_set_split_event")
 
     def workspace_bytes(self) -> int:
         return int(_lib().eb_sampler_workspace_bytes(self._h))

@@ -53,6 +53,7 @@ struct eb_sampler {
   int32_t* sample = nullptr;
   float* pmax = nullptr;
   int last_step = -1;
+  cudaEvent_t split_event = nullptr;  // recorded between the two kernels when set
 };
 
 namespace {
@@ -312,6 +313,8 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
       cudaSuccess)
     return EB_ERR_CUDA;
 
+  if (h->split_event && cudaEventRecord(h->split_event, st) != cudaSuccess) return EB_ERR_CUDA;
+
   const KernelCfg& kf = h->fin[dtype];
   const int32_t* act_index = h->act_index;
   const int32_t* n_act = h->n_act;
@@ -414,6 +417,12 @@ int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int3
     return EB_ERR_CUDA;
   }
   h->last_step = next_step - 1;
+  return EB_OK;
+}
+
+int eb_sampler_set_split_event(eb_sampler_t* h, void* event) {
+  if (!h) return EB_ERR_INVALID_ARG;
+  h->split_event = static_cast<cudaEvent_t>(event);
   return EB_OK;
 }
 

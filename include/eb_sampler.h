@@ -173,6 +173,15 @@ int eb_sampler_draws(eb_sampler_t* h, int32_t* sample, float* pmax, void* stream
 int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int32_t* stable,
                          int next_step, void* stream);
 
+/* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
+   the caller) is non-NULL, every following eb_sampler_step records it on
+   its stream between the step's two kernels, so that the caller can time
+   them apart with events recorded before and after the call.  Recording it
+   keeps the second kernel from starting early (programmatic dependent
+   launch), so set it only for timing; NULL turns it off.  No counterpart in
+   the method: it measures the implementation. */
+int eb_sampler_set_split_event(eb_sampler_t* h, void* event);
+
 /* Bytes of device workspace the handle holds. */
 size_t eb_sampler_workspace_bytes(const eb_sampler_t* h);
 
