@@ -14,6 +14,8 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <functional>
+#include <mutex>
 #include <new>
 
 #include "eb_finish.cuh"
@@ -454,3 +456,173 @@ const char* eb_strerror(int code) {
 int eb_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free row statistics (eb_row_stats_noalloc)
+//
+// For callers that cannot or must not allocate device memory (a hard memory
+// budget, a plugin given raw pointers, no sampler handle): the stream pass's
+// partial records live in a static device array instead of a workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocCtrlBytes = 256;  // stop flag, status, active index, count
+constexpr int kNoAllocMaxDevices = 64;
+
+}  // namespace
+
+// Scratch: [0, 256) control words (must start at zero: the stop flag of the
+// single pseudo-canvas and the status word; the active index and count are
+// written by the stream kernel), then the partial records.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[EB_NOALLOC_SCRATCH_BYTES];
+
+namespace ebk {
+
+// One 8-lane subgroup per row: the finish kernel's per-position reduction
+// (record merge, exact top group), without the draw and the canvas epilogue.
+template <int DT>
+__global__ void __launch_bounds__(256) row_stats_kernel(const StepArgs a,
+                                                        const int32_t* n_act_ptr) {
+  constexpr int kTPR = 8;
+  const int tid = threadIdx.x;
+  const int row = blockIdx.x * (256 / kTPR) + tid / kTPR;
+  const int sl = tid % kTPR;
+  const bool valid = row < a.L;
+  const unsigned long long NG =
+      (unsigned long long)(*n_act_ptr) * (unsigned long long)a.L * (unsigned long long)a.ng;
+  const RowOut ro = finish_row<DT, kTPR>(a, 0, 0, valid ? row : 0, valid, false, sl, NG);
+  if (valid && sl == 0) {
+    a.H_out[row] = ro.H;
+    a.amax_out[row] = ro.amax;
+  }
+}
+
+}  // namespace ebk
+
+namespace {
+
+struct NoAllocDevice {
+  std::once_flag once;
+  int rc = EB_ERR_CUDA;
+  unsigned char* scratch = nullptr;
+  int sms = 0;
+};
+NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+
+// Once per device: the scratch's device address and the stream kernel's
+// shared-memory opt-in (set to the device maximum, so that it never lowers
+// a value a sampler handle set for a larger active list).
+void noalloc_setup(NoAllocDevice& d, int device) {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    d.rc = EB_ERR_CUDA;
+    return;
+  }
+  int sms = 0, optin = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess) {
+    d.rc = EB_ERR_CUDA;
+    return;
+  }
+  if (major != 10) {
+    d.rc = EB_ERR_UNSUPPORTED;
+    return;
+  }
+  if ((size_t)optin < ebk::stream_layout<ebk::kF32>(1).total ||
+      (size_t)optin < ebk::stream_layout<ebk::kBF16>(1).total) {
+    d.rc = EB_ERR_OVERFLOW;
+    return;
+  }
+  if (cudaFuncSetAttribute(ebk::stream_kernel<ebk::kF32>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::stream_kernel<ebk::kBF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
+    d.rc = EB_ERR_CUDA;
+    return;
+  }
+  d.scratch = static_cast<unsigned char*>(p);
+  d.sms = sms;
+  d.rc = EB_OK;
+}
+
+template <int DT>
+int noalloc_launch(const NoAllocDevice& d, const void* logits, int32_t rows, int32_t V,
+                   double T, float* entropies, int32_t* argmax, cudaStream_t st) {
+  using Sh = ebk::StreamShape<DT>;
+  const int ng = (int)(((int64_t)V + ebk::kGroup - 1) / ebk::kGroup);
+  const uint64_t groups = (uint64_t)rows * (uint64_t)ng;
+  const uint64_t want = (groups + Sh::kStageGroups - 1) / Sh::kStageGroups;
+  const int grid = (int)std::min<uint64_t>((uint64_t)d.sms, std::max<uint64_t>(1, want));
+  // stream CTAs a row can meet (each CTA owns at least floor(groups / grid))
+  const uint64_t segs = ((uint64_t)(ng - 1) * (uint64_t)grid) / groups + 2;
+  const int max_segs = (int)std::min<uint64_t>((uint64_t)grid, segs);
+  const int nw = ebk::stream_consumer_warps();
+  const uint64_t rec_bytes =
+      (uint64_t)rows * (uint64_t)max_segs * (uint64_t)nw * (uint64_t)sizeof(Partial);
+  if (rec_bytes > EB_NOALLOC_SCRATCH_BYTES - kNoAllocCtrlBytes) return EB_ERR_OVERFLOW;
+
+  unsigned char* ctrl = d.scratch;
+  if (cudaMemsetAsync(ctrl, 0, kNoAllocCtrlBytes, st) != cudaSuccess) return EB_ERR_CUDA;
+  StepArgs a;
+  std::memset(&a, 0, sizeof(a));
+  a.logits = logits;
+  a.H_out = entropies;
+  a.amax_out = argmax;
+  a.stop_flags = ctrl;                                         // one pseudo-canvas, active
+  a.status = reinterpret_cast<uint32_t*>(ctrl + 4);
+  a.act_index = reinterpret_cast<int32_t*>(ctrl + 8);
+  a.n_act = reinterpret_cast<int32_t*>(ctrl + 12);
+  a.partials = reinterpret_cast<Partial*>(d.scratch + kNoAllocCtrlBytes);
+  a.B = 1;
+  a.L = rows;  // the rows are the positions of one pseudo-canvas
+  a.V = V;
+  a.ng = ng;
+  a.s = 0;
+  a.N = 1;
+  a.max_segs = max_segs;
+  a.nw = nw;
+  a.G1 = grid;
+  const size_t elt = DT == ebk::kF32 ? 4 : 2;
+  a.vec_ok = ((uintptr_t)logits % 16 == 0) && (((size_t)V * elt) % 16 == 0) ? 1 : 0;
+  a.greedy = 1;  // no draw: the stream pass skips the Gumbel race
+  a.c2 = (float)(1.4426950408889634 / T);
+  a.iT = (float)(1.0 / T);
+  void* args[] = {&a};
+  if (cudaLaunchKernel(reinterpret_cast<const void*>(&ebk::stream_kernel<DT>), dim3(grid),
+                       dim3(Sh::kThreads), args, ebk::stream_layout<DT>(1).total, st) !=
+      cudaSuccess)
+    return EB_ERR_CUDA;
+  const int32_t* n_act = a.n_act;
+  void* rargs[] = {&a, &n_act};
+  if (cudaLaunchKernel(reinterpret_cast<const void*>(&ebk::row_stats_kernel<DT>),
+                       dim3((unsigned)((rows + 31) / 32)), dim3(256), rargs, 0, st) !=
+      cudaSuccess)
+    return EB_ERR_CUDA;
+  return EB_OK;
+}
+
+}  // namespace
+
+extern "C" int eb_row_stats_noalloc(const void* logits, int dtype, int32_t rows, int32_t V,
+                                    double temperature, float* entropies, int32_t* argmax,
+                                    void* stream) {
+  if (!logits || !entropies || !argmax || rows < 1 || V < 1) return EB_ERR_INVALID_ARG;
+  if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
+  if (!(temperature > 0.0) || !std::isfinite(temperature)) return EB_ERR_INVALID_ARG;
+  if ((uintptr_t)logits % (dtype == EB_F32 ? 4u : 2u) != 0) return EB_ERR_INVALID_ARG;
+  if ((uint64_t)rows * (((uint64_t)V + ebk::kGroup - 1) / ebk::kGroup) >= (1ull << 46))
+    return EB_ERR_OVERFLOW;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return EB_ERR_CUDA;
+  if (device < 0 || device >= kNoAllocMaxDevices) return EB_ERR_UNSUPPORTED;
+  NoAllocDevice& d = g_noalloc_dev[device];
+  std::call_once(d.once, noalloc_setup, std::ref(d), device);
+  if (d.rc != EB_OK) return d.rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  return dtype == EB_F32
+             ? noalloc_launch<ebk::kF32>(d, logits, rows, V, temperature, entropies, argmax, st)
+             : noalloc_launch<ebk::kBF16>(d, logits, rows, V, temperature, entropies, argmax, st);
+}

@@ -173,6 +173,39 @@ int eb_sampler_draws(eb_sampler_t* h, int32_t* sample, float* pmax, void* stream
 int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int32_t* stable,
                          int next_step, void* stream);
 
+/* Allocation-free per-row statistics.  For `rows` rows of `V` logits
+   (dtype EB_F32 / EB_BF16, [rows][V] row-major, device memory, caller-owned)
+   writes each row's entropy in nats of softmax(z / temperature) into
+   `entropies` ([rows] fp32, device) and its argmax (lowest index on ties)
+   into `argmax` ([rows] int32, device), enqueued on `stream`.  These are the
+   entropies and argmax that eb_sampler_step computes for a position at the
+   same temperature (bit for bit when the sampler's L lies in 129 .. 256, so
+   that both use the same per-position lane count).
+
+   For callers that cannot allocate device memory, or must not: code that
+   runs under a hard device-memory budget, a plugin handed raw pointers by a
+   host that owns the allocator, or a caller that has no eb_sampler_t
+   (eb_sampler_init allocates its workspace).  This call allocates nothing:
+   its scratch (the per-(row, SM, warp) partial records of the stream pass)
+   is a static device array of EB_NOALLOC_SCRATCH_BYTES bytes in the
+   library, looked up once per device.
+     - The first call on a device performs that one-time setup (symbol
+       lookup, kernel attributes); make it before any stream capture.
+     - Sizes beyond the scratch return EB_ERR_OVERFLOW: rows x (stream CTAs
+       a row can span) x 12 records x 32 bytes must fit (e.g. up to 8192
+       rows of 262144 logits).
+     - Calls that overlap in time (different streams or threads) share the
+       scratch and race; serialise them.
+   Non-finite softmax sums set bit EB_STATUS_NONFINITE of the scratch status
+   word, which is cleared at the start of every call and not otherwise
+   reported.  Returns EB_ERR_INVALID_ARG for NULL pointers, rows or V < 1, a
+   temperature that is not finite and positive, or logits not aligned to
+   their element size.  No counterpart in the DiffusionGemma pages: it
+   exposes the sampler's row reduction on its own, for deployment. */
+#define EB_NOALLOC_SCRATCH_BYTES (8u << 20)
+int eb_row_stats_noalloc(const void* logits, int dtype, int32_t rows, int32_t V,
+                         double temperature, float* entropies, int32_t* argmax, void* stream);
+
 /* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
    the caller) is non-NULL, every following eb_sampler_step records it on
    its stream between the step's two kernels, so that the caller can time
