@@ -231,6 +231,25 @@ struct GroupIO<kBF16> {
     const uint32_t m = bf16x2_max(bf16x2_max(t[0], t[1]), bf16x2_max(t[2], t[3]));
     return fmaxf(bf16_lo(m), bf16_hi(m));
   }
+  __device__ __forceinline__ static void exp1_of(const unsigned char* g0, int rot, float c2,
+                                                 float r0, float& S0, float& W0) {
+    const uint4* q0 = reinterpret_cast<const uint4*>(g0);
+    const float2 c2v = make_float2(c2, c2);
+    const float2 n0 = make_float2(-r0 * c2, -r0 * c2);
+    float2 s0[4], w0[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s0[i] = w0[i] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint4 a = q0[(k + rot) & 7];
+      const uint32_t wa[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        acc_pair(make_float2(bf16_lo(wa[i]), bf16_hi(wa[i])), c2v, n0, s0[i], w0[i]);
+    }
+    S0 = sum4(s0);
+    W0 = sum4(w0);
+  }
   // Exponential pass of two groups at once (independent chains interleave).
   __device__ __forceinline__ static void exp2_of(const unsigned char* g0, const unsigned char* g1,
                                                  int rot, float c2, float r0, float r1,
@@ -265,6 +284,23 @@ struct GroupIO<kBF16> {
 
 template <>
 struct GroupIO<kF32> {
+  __device__ __forceinline__ static void exp1_of(const unsigned char* g0, int rot, float c2,
+                                                 float r0, float& S0, float& W0) {
+    const float4* q0 = reinterpret_cast<const float4*>(g0);
+    const float2 c2v = make_float2(c2, c2);
+    const float2 n0 = make_float2(-r0 * c2, -r0 * c2);
+    float2 s0[4], w0[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) s0[i] = w0[i] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float4 a = q0[(k + rot) & 15];
+      acc_pair(make_float2(a.x, a.y), c2v, n0, s0[(2 * k) & 3], w0[(2 * k) & 3]);
+      acc_pair(make_float2(a.z, a.w), c2v, n0, s0[(2 * k + 1) & 3], w0[(2 * k + 1) & 3]);
+    }
+    S0 = sum4(s0);
+    W0 = sum4(w0);
+  }
   static constexpr int kPieces = 16;
   __device__ __forceinline__ static float max_of(const unsigned char* gp, int rot) {
     const float4* q = reinterpret_cast<const float4*>(gp);

@@ -44,11 +44,12 @@ struct FinCtrl {
   int stable_prev;
   double dscr[kFinWarps];
   int iscr[kFinWarps];
+  int cscr[kFinWarps];
   unsigned long long uscr[kFinWarps];
 };
 
 struct FinLayout {
-  uint32_t ctrl, H, am, smp, pm, prev, tok, open, pick, keys, skeys, total;
+  uint32_t ctrl, H, am, smp, pm, prev, tok, open, pick, keys, total;
 };
 
 __host__ __device__ inline FinLayout fin_layout(int L) {
@@ -58,8 +59,6 @@ __host__ __device__ inline FinLayout fin_layout(int L) {
   y.ctrl = o;
   o += (uint32_t)((sizeof(FinCtrl) + 15) / 16 * 16);
   y.keys = o;
-  o += 8u * l;
-  y.skeys = o;
   o += 8u * l;
   y.H = o;
   o += 4u * l;
@@ -93,18 +92,6 @@ __host__ __device__ inline int fin_lanes_per_row(int L) {
 // ---------------------------------------------------------------------------
 // 256-thread block helpers (whole CTA, __syncthreads)
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ double fin_block_sum(double v, FinCtrl* c) {
-  const int tid = threadIdx.x;
-#pragma unroll
-  for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  if ((tid & 31) == 0) c->dscr[tid >> 5] = v;
-  __syncthreads();
-  double r = 0.0;
-  for (int w = 0; w < kFinWarps; ++w) r += c->dscr[w];
-  __syncthreads();
-  return r;
-}
-
 __device__ __forceinline__ int fin_block_sum_int(int v, FinCtrl* c) {
   const int tid = threadIdx.x;
 #pragma unroll
@@ -130,27 +117,6 @@ __device__ __forceinline__ unsigned long long fin_block_min(unsigned long long v
   for (int w = 1; w < kFinWarps; ++w) r = c->uscr[w] < r ? c->uscr[w] : r;
   __syncthreads();
   return r;
-}
-
-// Exclusive prefix of v over the CTA; *total gets the sum.
-__device__ __forceinline__ int fin_excl_scan(int v, FinCtrl* c, int* total) {
-  const int tid = threadIdx.x, lane = tid & 31;
-  int x = v;
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const int y = __shfl_up_sync(0xffffffffu, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) c->iscr[tid >> 5] = x;
-  __syncthreads();
-  int off = 0, tot = 0;
-  for (int w = 0; w < kFinWarps; ++w) {
-    if (w < (tid >> 5)) off += c->iscr[w];
-    tot += c->iscr[w];
-  }
-  __syncthreads();
-  *total = tot;
-  return off + x - v;
 }
 
 // Sort keys: ascending (H, l) (H >= 0, so its float bits order like the
@@ -226,9 +192,24 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
     const int c_last = cta_of(g_first + (unsigned long long)a.ng - 1ull, NG, a.G1);
     const int nrec = (c_last - c_first + 1) * a.nw;
     const Partial* rec = a.partials + grow * (size_t)(a.max_segs * a.nw);
-    for (int i = sl; i < nrec; i += TPR) {
-      const int c = c_first + i / a.nw;
-      if (range_start(c, NG, a.G1) < range_start(c + 1, NG, a.G1)) merge(R, rec[i], a.c2);
+    if (NG >= (unsigned long long)a.G1) {
+      // every stream CTA owns at least one group, so every CTA from c_first
+      // to c_last wrote its records for this row: load four at a time
+      for (int i0 = sl; i0 < nrec; i0 += 4 * TPR) {
+        Partial q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int i = i0 + u * TPR;
+          q[u] = i < nrec ? rec[i] : empty_partial();
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) merge(R, q[u], a.c2);
+      }
+    } else {
+      for (int i = sl; i < nrec; i += TPR) {
+        const int c = c_first + i / a.nw;
+        if (range_start(c, NG, a.G1) < range_start(c + 1, NG, a.G1)) merge(R, rec[i], a.c2);
+      }
     }
   }
 #pragma unroll
@@ -377,16 +358,57 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
 // ---------------------------------------------------------------------------
 // Canvas epilogue (cluster rank 0, 256 threads, values in shared memory)
 // ---------------------------------------------------------------------------
+// One block-wide pass: sum of a (double), OR of b, exclusive prefix of c
+// (*c_total gets the sum of c).
+__device__ __forceinline__ void fin_block_reduce(double& a, int& b, int& c, int* c_total,
+                                                 FinCtrl* ctrl) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  double x = a;
+  int y = b, z = c;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y |= __shfl_xor_sync(0xffffffffu, y, o);
+  }
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(0xffffffffu, z, o);
+    if (lane >= o) z += t;
+  }
+  if (lane == 31) {
+    ctrl->dscr[warp] = x;
+    ctrl->iscr[warp] = y;
+    ctrl->cscr[warp] = z;
+  }
+  __syncthreads();
+  double sx = 0.0;
+  int sy = 0, off = 0, tot = 0;
+#pragma unroll
+  for (int w = 0; w < kFinWarps; ++w) {
+    sx += ctrl->dscr[w];
+    sy |= ctrl->iscr[w];
+    if (w < warp) off += ctrl->cscr[w];
+    tot += ctrl->cscr[w];
+  }
+  __syncthreads();
+  a = sx;
+  b = sy;
+  c = off + z - c;
+  *c_total = tot;
+}
+
 __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const float* sH,
                                 const int* sAm, const int* sSmp, const float* sPm,
                                 const int* sPrev, const int* sTok, const uint8_t* sOpen,
-                                uint8_t* pick, unsigned long long* keys,
-                                unsigned long long* skeys) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+                                uint8_t* pick, unsigned long long* keys) {
+  const int tid = threadIdx.x;
   const int L = a.L;
   const size_t row0 = (size_t)bi * (size_t)L;
   const bool br = a.rule == kRuleBR;
 
+  // pass 1: entropy sum, argmax stability, candidates (EB: open with
+  // H <= gamma, no other can be in the prefix; BR: open below the threshold,
+  // which compete for the quota, while those at or above it commit outright)
   double sumH = 0.0;
   int neq = a.s < 1 ? 1 : 0;
   int ncand = 0;
@@ -403,19 +425,15 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
       ++ncand;
     }
   }
-  const double totH = fin_block_sum(sumH, ctrl);
-  const int any_neq = fin_block_sum_int(neq, ctrl);
-  const int stable_new = any_neq ? 0 : ctrl->stable_prev + 1;
-  const double meanH = totH / (double)L;
+  int n_c = 0;
+  int pos = ncand;
+  fin_block_reduce(sumH, neq, pos, &n_c, ctrl);
+  const int stable_new = neq ? 0 : ctrl->stable_prev + 1;
+  const double meanH = sumH / (double)L;
   const bool fired = a.stop_enabled && stable_new >= a.stability_steps && meanH < a.tau;
   const bool last_step = a.s == a.N - 1;
 
   if (!fired) {
-    // Candidates.  EB: open positions with H <= gamma (no other can be in
-    // the prefix).  BR: open positions below the threshold compete for the
-    // quota; those at or above it are committed outright.
-    int n_c = 0;
-    int pos = fin_excl_scan(ncand, ctrl, &n_c);
     for (int l = tid; l < L; l += kFinThreads) {
       if (!sOpen[l]) continue;
       if (!br) {
@@ -427,60 +445,42 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
       }
     }
     __syncthreads();
+    // EB: candidate c is in the lowest-entropy prefix iff the entropies of all
+    // candidates at or before it in (H, l) order sum to <= gamma (the sums
+    // grow along the order).  BR: the quota goes to the first candidates in
+    // (-pmax, l) order.
     for (int c = tid; c < n_c; c += kFinThreads) {
       const unsigned long long kc = keys[c];
-      int rank = 0;
+      if (!br) {
+        double cum = (double)__uint_as_float((uint32_t)(kc >> 32));
+        for (int j = 0; j < n_c; ++j) {
+          const unsigned long long kj = keys[j];
+          if (kj < kc) cum += (double)__uint_as_float((uint32_t)(kj >> 32));
+        }
+        if (cum <= a.gamma) pick[(int)(kc & 0xffffffffu)] = 1;
+      } else {
+        int rank = 0;
 #pragma unroll 4
-      for (int j = 0; j < n_c; ++j) rank += keys[j] < kc;
-      if (!br) skeys[rank] = kc;
-      else if (rank < a.quota) pick[(int)(kc & 0xffffffffu)] = 1;
+        for (int j = 0; j < n_c; ++j) rank += keys[j] < kc;
+        if (rank < a.quota) pick[(int)(kc & 0xffffffffu)] = 1;
+      }
     }
     __syncthreads();
-    if (!br) {
-      // longest prefix of the sorted candidates with cumulative H <= gamma
-      if (warp == 0) {
-        const int chunk = (n_c + 31) / 32;
-        const int lo = lane * chunk;
-        const int hi = lo + chunk < n_c ? lo + chunk : n_c;
-        double part = 0.0;
-        for (int i = lo; i < hi; ++i) part += (double)__uint_as_float((uint32_t)(skeys[i] >> 32));
-        double x = part;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-          const double y = __shfl_up_sync(0xffffffffu, x, o);
-          if (lane >= o) x += y;
-        }
-        double cum = x - part;
-        int cnt = 0;
-        for (int i = lo; i < hi; ++i) {
-          cum += (double)__uint_as_float((uint32_t)(skeys[i] >> 32));
-          if (cum <= a.gamma) ++cnt;
-          else break;
-        }
-#pragma unroll
-        for (int o = 16; o; o >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, o);
-        if (lane == 0) ctrl->kpref = cnt;
+    // EB with no candidate: the single lowest (H, l).  MI: the prefix plus
+    // the next open position in (H, l) order.  Candidates (H <= gamma) come
+    // before every other open position, so both are the lowest open
+    // position left out of the prefix.
+    if (!br && (a.rule == kRuleMI || n_c == 0)) {
+      unsigned long long best = ~0ull;
+      for (int l = tid; l < L; l += kFinThreads) {
+        if (!sOpen[l] || pick[l]) continue;
+        const unsigned long long kk = key_asc(sH[l], l);
+        best = kk < best ? kk : best;
       }
+      best = fin_block_min(best, ctrl);
+      if (tid == 0 && best != ~0ull) pick[(int)(best & 0xffffffffu)] = 1;
       __syncthreads();
-      const int kpref = ctrl->kpref;
-      for (int i = tid; i < kpref; i += kFinThreads) pick[(int)(skeys[i] & 0xffffffffu)] = 1;
-      // EB with an empty prefix: the single lowest (H, l).  MI: the prefix
-      // plus the next position in (H, l) order.
-      const bool mi = a.rule == kRuleMI;
-      if (mi && kpref < n_c) {
-        if (tid == 0) pick[(int)(skeys[kpref] & 0xffffffffu)] = 1;
-      } else if (kpref == 0 || mi) {
-        unsigned long long best = ~0ull;
-        for (int l = tid; l < L; l += kFinThreads) {
-          if (!sOpen[l] || (mi && (double)sH[l] <= a.gamma)) continue;
-          const unsigned long long kk = key_asc(sH[l], l);
-          best = kk < best ? kk : best;
-        }
-        best = fin_block_min(best, ctrl);
-        if (tid == 0 && best != ~0ull) pick[(int)(best & 0xffffffffu)] = 1;
-      }
     }
-    __syncthreads();
   }
 
   // commit, renoise, remember the argmax
@@ -590,8 +590,7 @@ __global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThread
                     reinterpret_cast<const float*>(smem + lay.pm),
                     reinterpret_cast<const int*>(smem + lay.prev),
                     reinterpret_cast<const int*>(smem + lay.tok), smem + lay.open,
-                    smem + lay.pick, reinterpret_cast<unsigned long long*>(smem + lay.keys),
-                    reinterpret_cast<unsigned long long*>(smem + lay.skeys));
+                    smem + lay.pick, reinterpret_cast<unsigned long long*>(smem + lay.keys));
 }
 
 // Initial canvas: uniform-random tokens (stream 2), nothing committed.

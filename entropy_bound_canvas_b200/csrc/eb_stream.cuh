@@ -36,22 +36,26 @@ namespace ebk {
 #ifndef EB_STREAM_STAGE_KB
 #define EB_STREAM_STAGE_KB 32
 #endif
+#ifndef EB_STREAM_GROUPS_PER_LANE
+#define EB_STREAM_GROUPS_PER_LANE 2
+#endif
 
 constexpr int kStages = EB_STREAM_STAGES;
 
-// Shape of the stream CTA: kConsumerWarps consumer warps + 1 producer warp,
+// Shape of the stream CTA: kConsumerWarps consumer warps + 2 producer warps,
 // a ring of kStages stages of kStageBytes each (192 KB with the defaults:
 // one CTA per SM).  Twelve consumer warps, each lane reducing two groups at
 // a time, keep the SM's MUFU and FMA pipes busy.
 template <int DT>
 struct StreamShape {
   static constexpr int kConsumerWarps = EB_STREAM_CONSUMER_WARPS;
-  static constexpr int kThreads = (kConsumerWarps + 1) * 32;
+  static constexpr int kThreads = (kConsumerWarps + 2) * 32;  // + copy and word producers
   static constexpr int kStageBytes = EB_STREAM_STAGE_KB * 1024;
   // room for a copy widened to 16-byte boundaries; 128-byte aligned stages
   static constexpr int kStageStride = kStageBytes + 128;
   static constexpr int kStageGroups = kStageBytes / (kGroup * elt_bytes(DT));
-  static constexpr int kSubGroups = 64;  // groups per sub-tile: two per lane
+  static constexpr int kGroupsPerLane = EB_STREAM_GROUPS_PER_LANE;
+  static constexpr int kSubGroups = 32 * kGroupsPerLane;  // groups per sub-tile
   static constexpr int kSubPerStage = kStageGroups / kSubGroups;
   static_assert(kSubPerStage >= 1 && (kSubPerStage & (kSubPerStage - 1)) == 0,
                 "sub-tiles per stage must be a power of two");
@@ -195,14 +199,9 @@ __device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int 
   return base;
 }
 
-#ifndef EB_STREAM_MAXNREG
-#define EB_STREAM_MAXNREG 128
-#endif
-
-// 128 registers keep the two-group consumer loop free of spills; with 12
-// consumer warps the CTA then holds 53 K of the SM's 64 K registers.
+// One CTA per SM: the register cap is the register file over the block.
 template <int DT>
-__global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
+__global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(const StepArgs a) {
   using Sh = StreamShape<DT>;
   using IO = GroupIO<DT>;
   extern __shared__ __align__(128) unsigned char smem[];
@@ -248,44 +247,39 @@ __global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
   const char* logits = reinterpret_cast<const char*>(a.logits);
 
   if (warp == Sh::kConsumerWarps) {
-    // ------------------------------------------------------------ producer
-    const uint64_t policy = evict_first_policy();
-    TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kStageGroups);
-    Tile t;
-    int k = 0, st = 0;
-    uint32_t ph = 0;  // parity of the current pass over the ring
-    long long row_seen = -1;
-    int bi = 0, samp = 0;
-    while (it.next(t)) {
-      if (k >= kStages) {
-        int ok = 1;
-        if (lane == 0) ok = mbar_wait(&empty[st], ph ^ 1u) ? 1 : 0;
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          if (lane == 0) {
-            atomicOr(a.status, kStatusTimeout);
-            *(volatile int*)&ctrl->abort = 1;
-          }
+    // ------------------------------------------------------- copy producer
+    // Lane 0 alone: waits for a free stage, writes the tile's description
+    // and issues its bulk copy (the stage's first arrival, with the bytes).
+    if (lane == 0) {
+      const uint64_t policy = evict_first_policy();
+      TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kStageGroups);
+      Tile t;
+      int k = 0, st = 0;
+      uint32_t ph = 0;  // parity of the current pass over the ring
+      long long row_seen = -1;
+      int bi = 0, samp = 0;
+      while (it.next(t)) {
+        if (k >= kStages && !mbar_wait(&empty[st], ph ^ 1u)) {
+          atomicOr(a.status, kStatusTimeout);
+          *(volatile int*)&ctrl->abort = 1;
           break;
         }
-      }
-      if (*(volatile int*)&ctrl->abort) break;
-      if (t.r != row_seen) {
-        row_seen = t.r;
-        bi = act[t.ai];
-        samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
-      }
-      const char* src = logits + ((size_t)bi * (size_t)a.L + (size_t)t.l) * row_bytes +
-                        (size_t)t.j0 * kGroup * elt_bytes(DT);
-      size_t nel = (size_t)t.cnt * kGroup;
-      if ((size_t)t.j0 * kGroup + nel > (size_t)a.V) nel = (size_t)a.V - (size_t)t.j0 * kGroup;
-      // The copy is widened to 16-byte boundaries: at most 15 bytes on each
-      // side, inside the 16-byte blocks that hold the tile's first and last
-      // logits.
-      const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~(uintptr_t)15;
-      const uintptr_t a1 =
-          (reinterpret_cast<uintptr_t>(src) + nel * elt_bytes(DT) + 15) & ~(uintptr_t)15;
-      if (lane == 0) {
+        if (*(volatile int*)&ctrl->abort) break;
+        if (t.r != row_seen) {
+          row_seen = t.r;
+          bi = act[t.ai];
+          samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
+        }
+        const char* src = logits + ((size_t)bi * (size_t)a.L + (size_t)t.l) * row_bytes +
+                          (size_t)t.j0 * kGroup * elt_bytes(DT);
+        size_t nel = (size_t)t.cnt * kGroup;
+        if ((size_t)t.j0 * kGroup + nel > (size_t)a.V) nel = (size_t)a.V - (size_t)t.j0 * kGroup;
+        // The copy is widened to 16-byte boundaries: at most 15 bytes on each
+        // side, inside the 16-byte blocks that hold the tile's first and last
+        // logits.
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~(uintptr_t)15;
+        const uintptr_t a1 =
+            (reinterpret_cast<uintptr_t>(src) + nel * elt_bytes(DT) + 15) & ~(uintptr_t)15;
         TileMeta m;
         m.r = (int)t.r;
         m.j0 = t.j0;
@@ -299,30 +293,54 @@ __global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
         mbar_arrive_expect_tx(&full[st], (uint32_t)(a1 - a0));
         bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
                   (uint32_t)(a1 - a0), &full[st], policy);
+        st_release_shared(&ctrl->issued, k + 1);
+        ++k;
+        if (++st == kStages) {
+          st = 0;
+          ph ^= 1u;
+        }
       }
-      if (samp) {  // while the copy is in flight: the tile's group-stream words
+    }
+  } else if (warp == Sh::kConsumerWarps + 1) {
+    // ------------------------------------------------------- word producer
+    // Follows the copy producer: once tile k is issued (so its stage is free
+    // and its description written), computes the group-stream Philox words
+    // of an open position's groups into the stage's header and makes the
+    // stage's second arrival.  Kept off the copy producer so that copies are
+    // never issued late.
+    const int n_tiles = ctrl->n_sub / Sh::kSubPerStage;
+    int st = 0, words_done = 0;
+    for (int k = 0; k < n_tiles; ++k, words_done = k) {
+      if (!wait_counter_above(&ctrl->issued, k)) {
+        if (lane == 0) {
+          atomicOr(a.status, kStatusTimeout);
+          *(volatile int*)&ctrl->abort = 1;
+        }
+        break;
+      }
+      const TileMeta m = meta[st];
+      if (m.sampling) {
         uint32_t* wd = words + st * Sh::kStageGroups;
-        const int c0 = t.j0 >> 2, c1 = (t.j0 + t.cnt - 1) >> 2;
-        const uint32_t c3 = (uint32_t)(a.canvas_offset + bi) | (kStreamGroup << 24);
+        const int c0 = m.j0 >> 2, c1 = (m.j0 + m.cnt - 1) >> 2;
+        const uint32_t c3 = (uint32_t)(a.canvas_offset + m.bi) | (kStreamGroup << 24);
         for (int c = c0 + lane; c <= c1; c += 32) {
-          const Words4 w = philox((uint32_t)c, (uint32_t)t.l, (uint32_t)a.s, c3, a.key0, a.key1);
+          const Words4 w = philox((uint32_t)c, (uint32_t)m.l, (uint32_t)a.s, c3, a.key0, a.key1);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int j = 4 * c + q - t.j0;
-            if (j >= 0 && j < t.cnt) wd[j] = w.w[q];
+            const int j = 4 * c + q - m.j0;
+            if (j >= 0 && j < m.cnt) wd[j] = w.w[q];
           }
         }
       }
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&full[st]);  // header (meta, words) complete
-        st_release_shared(&ctrl->issued, k + 1);
-      }
-      ++k;
-      if (++st == kStages) {
-        st = 0;
-        ph ^= 1u;
-      }
+      if (lane == 0) mbar_arrive(&full[st]);  // header (words) complete
+      if (++st == kStages) st = 0;
+    }
+    // After an abort: the second arrival of every tile already issued, so
+    // that the drain below sees each copy complete.
+    if (lane == 0 && *(volatile int*)&ctrl->abort) {
+      const int issued = ld_acquire_shared(&ctrl->issued);
+      for (int k = words_done; k < issued; ++k) mbar_arrive(&full[k % kStages]);
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -390,7 +408,7 @@ __global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
       }
       const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
       if (sub * Sh::kSubGroups < m.cnt) {  // warp-uniform
-        const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
+        const bool has0 = gl0 < m.cnt, has1 = Sh::kGroupsPerLane == 2 && gl1 < m.cnt;
         const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
         const unsigned char* gp0 = sbase + (size_t)(has0 ? gl0 : 0) * kGroup * elt_bytes(DT);
         const unsigned char* gp1 = has1 ? sbase + (size_t)gl1 * kGroup * elt_bytes(DT) : gp0;
@@ -401,7 +419,7 @@ __global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
         float mg0, mg1;
         if (fast) {
           mg0 = IO::max_of(gp0, rot);
-          mg1 = IO::max_of(gp1, rot);
+          mg1 = Sh::kGroupsPerLane == 2 ? IO::max_of(gp1, rot) : -INFINITY;
         } else {
           mg0 = has0 ? group_max_safe<DT>(gp0, len0) : -INFINITY;
           mg1 = has1 ? group_max_safe<DT>(gp1, len1) : -INFINITY;
@@ -411,14 +429,18 @@ __global__ void __maxnreg__(EB_STREAM_MAXNREG) stream_kernel(const StepArgs a) {
         warp_raise(A, fmaxf(mg0, mg1), mg0 >= mg1 ? j0 : j1, a.c2);
         float S0 = 0.f, W0 = 0.f, S1 = 0.f, W1 = 0.f;
         if (fast) {
-          IO::exp2_of(gp0, gp1, rot, a.c2, A.M, A.M, S0, W0, S1, W1);
+          if constexpr (Sh::kGroupsPerLane == 2) {
+            IO::exp2_of(gp0, gp1, rot, a.c2, A.M, A.M, S0, W0, S1, W1);
+          } else {
+            IO::exp1_of(gp0, rot, a.c2, A.M, S0, W0);
+          }
           // -inf (or other non-finite) logits: redo the group term by term
           if (!(W0 >= -3.0e38f)) {
             const float2 q = group_sums_safe<DT>(gp0, kGroup, a.c2, A.M);
             S0 = q.x;
             W0 = q.y;
           }
-          if (!(W1 >= -3.0e38f)) {
+          if (has1 && !(W1 >= -3.0e38f)) {
             const float2 q = group_sums_safe<DT>(gp1, kGroup, a.c2, A.M);
             S1 = q.x;
             W1 = q.y;
