@@ -56,8 +56,9 @@ def make_sampler(E, w, **over):
     return E.EBSampler(w.B, w.L, w.V, device=DEV, **cfg)
 
 
-def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=3):
-    """Whole trajectory, every canvas, every position compared with the oracle."""
+def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=3, mask=None):
+    """Whole trajectory, every canvas, every position compared with the oracle.
+    `mask(logits, s)` may edit the generated logits in place (e.g. -inf)."""
     eb = make_sampler(E, w, canvas_offset=canvas_offset)
     canvas, committed, stop = eb.new_canvas()
     H, amax = eb.outputs()
@@ -71,6 +72,8 @@ def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=3):
     prev_H = None
     for s in range(w.num_steps):
         synth.generate_device(w, s, logits, b0=canvas_offset)
+        if mask is not None:
+            mask(logits, s)
         eb.step(logits, s, canvas, committed, H, amax, stop)
         smp, pm = eb.draws()
         torch.cuda.synchronize()
@@ -121,6 +124,54 @@ MID = synth.WORKLOADS["canvas"].replace(name="mid", B=3, L=64, V=8232, num_steps
 def test_full_parity(E, name, w):
     stats = run_full(E, w)
     print(name, stats)
+
+
+def _mask_neg_inf(V):
+    """-inf logits, as a vocabulary mask would leave them: a random tenth of the
+    vocabulary (new each step), one whole 64-logit group, and the last logit."""
+    def apply(logits, s):
+        g = torch.Generator(device="cpu").manual_seed(1000 + s)
+        m = torch.rand(V, generator=g) < 0.1
+        m[3 * 64:4 * 64] = True
+        m[V - 1] = True
+        logits[:, :, m.to(logits.device)] = float("-inf")
+    return apply
+
+
+@pytest.mark.parametrize("name,w", [
+    ("masked_bf16", MID.replace(B=2, num_steps=12, seed=21)),
+    ("masked_f32", MID.replace(B=2, num_steps=12, seed=22, dtype=synth.F32)),
+    ("masked_unaligned_bf16", MID.replace(B=2, num_steps=8, seed=23, V=5001)),
+])
+def test_full_parity_neg_inf_logits(E, name, w):
+    """Masked (-inf) logits contribute nothing to the entropy, never win a
+    draw, and never become the argmax, exactly as in the oracle."""
+    stats = run_full(E, w, mask=_mask_neg_inf(w.V))
+    print(name, stats)
+
+
+def test_split_event_times_the_two_kernels(E):
+    w = MID.replace(B=1, num_steps=4)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    logits = alloc_logits(w)
+    synth.generate_device(w, 0, logits)
+    H0 = None
+    for use in (False, True):
+        eb.init_canvas(canvas, committed, stop)
+        a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        eb.set_split_event(m if use else None)
+        a.record()
+        eb.step(logits, 0, canvas, committed, H, amax, stop)
+        b.record()
+        torch.cuda.synchronize()
+        if use:
+            assert a.elapsed_time(m) > 0 and m.elapsed_time(b) > 0
+            assert torch.equal(H, H0)  # recording the event changes no result
+        H0 = H.clone()
+    eb.set_split_event(None)
+    eb.close()
 
 
 def test_full_parity_unaligned_rows(E):
