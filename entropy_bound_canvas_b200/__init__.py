@@ -52,6 +52,7 @@ class Config(C.Structure):
         ("stability_steps", C.c_int32), ("rule", C.c_int32),
         ("threshold", C.c_double), ("quota", C.c_int32), ("greedy", C.c_int32),
         ("canvas_offset", C.c_int32), ("seed", C.c_uint64),
+        ("editing_threshold", C.c_double),
     ]
 
 

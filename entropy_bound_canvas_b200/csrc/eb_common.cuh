@@ -64,6 +64,7 @@ struct StepArgs {
   int canvas_offset;
   float c2, iT;
   double gamma, tau, theta;
+  double eps_edit;  // block refinement editing threshold; < 0: no editing
   uint32_t key0, key1;
 };
 

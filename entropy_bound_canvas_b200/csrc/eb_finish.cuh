@@ -486,8 +486,13 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
   // commit, renoise, remember the argmax
   const uint32_t bg = (uint32_t)(a.canvas_offset + bi);
   int left = 0;
+  const bool edit = !fired && a.eps_edit >= 0.0;
   for (int l = tid; l < L; l += kFinThreads) {
-    if (sOpen[l]) {
+    if (!sOpen[l]) {
+      // block refinement editing: a committed position whose argmax moved
+      // takes it when the argmax is confident enough
+      if (edit && sAm[l] != sTok[l] && (double)sPm[l] >= a.eps_edit) a.canvas[row0 + l] = sAm[l];
+    } else {
       if (fired) {
         a.canvas[row0 + l] = sAm[l];
         a.committed[row0 + l] = 1;

@@ -88,7 +88,8 @@ int validate_config(const eb_config_t* c) {
                       std::isfinite(c->t_min)))
     return EB_ERR_INVALID_ARG;
   if (!(c->entropy_bound >= 0.0) || !std::isfinite(c->entropy_bound)) return EB_ERR_INVALID_ARG;
-  if (std::isnan(c->stop_entropy) || std::isnan(c->threshold)) return EB_ERR_INVALID_ARG;
+  if (std::isnan(c->stop_entropy) || std::isnan(c->threshold) || std::isnan(c->editing_threshold))
+    return EB_ERR_INVALID_ARG;
   if (c->stability_steps < 0 || c->quota < 0) return EB_ERR_INVALID_ARG;
   // group numbering fits the 64-bit work split: B * L * ng * grid < 2^63
   const uint64_t ng = ((uint64_t)c->V + ebk::kGroup - 1) / ebk::kGroup;
@@ -155,6 +156,7 @@ void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V) {
   cfg->greedy = 0;
   cfg->canvas_offset = 0;
   cfg->seed = 0;
+  cfg->editing_threshold = -1.0;
 }
 
 int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
@@ -302,6 +304,7 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.gamma = c.entropy_bound;
   a.tau = c.stop_entropy;
   a.theta = c.threshold;
+  a.eps_edit = c.rule == EB_RULE_BLOCK_REFINEMENT ? c.editing_threshold : -1.0;
   a.key0 = (uint32_t)(c.seed & 0xffffffffu);
   a.key1 = (uint32_t)(c.seed >> 32);
 
@@ -453,7 +456,7 @@ const char* eb_strerror(int code) {
   }
 }
 
-int eb_version(void) { return 100; }
+int eb_version(void) { return 101; }
 
 }  // extern "C"
 

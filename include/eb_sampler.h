@@ -118,6 +118,13 @@ typedef struct {
   int32_t greedy;          /* 1: temperature 0.0 -- shape with T = 1, commit argmax, no draw */
   int32_t canvas_offset;   /* global index of canvas 0; offset + B <= 2^24 */
   uint64_t seed;           /* key of every Philox4x32-10 draw */
+  double editing_threshold; /* block refinement re-editing (diffusers "DiffusionGemma",
+                               Schedulers: editing_threshold lets the scheduler re-edit
+                               committed tokens).  Read here as: at a step where the stop
+                               did not fire, a position committed before the step takes
+                               this step's argmax when the argmax differs from its token
+                               and pmax >= editing_threshold; it stays committed.  < 0
+                               (the default) disables it; other rules ignore it.  Not NaN. */
 } eb_config_t;
 
 /* Fill *cfg with the model card's settings for B canvases of L x V. */

@@ -60,7 +60,7 @@ class _Config(C.Structure):
         ("stability_steps", C.c_int32), ("rule", C.c_int32),
         ("threshold", C.c_double), ("quota", C.c_int32), ("greedy", C.c_int32),
         ("group_size", C.c_int32), ("canvas_offset", C.c_int32),
-        ("seed", C.c_uint64),
+        ("seed", C.c_uint64), ("editing_threshold", C.c_double),
     ]
 
 
@@ -69,6 +69,7 @@ class Margins(C.Structure):
         ("cum_margin", C.c_double), ("cut_gap", C.c_double), ("stop_margin", C.c_double),
         ("br_margin", C.c_double), ("quota_gap", C.c_double), ("mean_H", C.c_double),
         ("n_commit", C.c_int32), ("fired", C.c_int32),
+        ("edit_margin", C.c_double), ("n_edit", C.c_int32), ("pad", C.c_int32),
     ]
 
     def as_dict(self):
@@ -94,6 +95,7 @@ class Config:
     group_size: int = 64
     canvas_offset: int = 0
     seed: int = 0
+    editing_threshold: float = -1.0
 
     def c(self) -> _Config:
         return _Config(**{f.name: getattr(self, f.name) for f in dataclasses.fields(self)})

@@ -264,7 +264,11 @@ static int cmp_key_desc(const void* a, const void* b) { /* (-key, l) ascending *
       EB_MI the same with the prefix's sum minus its largest entropy <= gamma
             (the "mutual information bound" wording of the model cards);
       BR    [DP-SCHED]: open positions with pmax >= threshold, plus the next
-            `quota` by (-pmax, l);
+            `quota` by (-pmax, l); with editing enabled, first, every position
+            committed before this step whose argmax differs from its token
+            takes the argmax when pmax >= editing_threshold ([DP-SCHED]:
+            editing_threshold lets the scheduler re-edit committed tokens;
+            the condition and the replacement token are this reading's);
    4. the last step (s = N-1) commits every remaining open position with its
       sampled token, stop = 3 (as the DDIM scheduler commits its predictions
       at the last step, [DP-SCHED]); if nothing is left open, stop = 2;
@@ -285,6 +289,9 @@ void ebo_canvas_decide(const ebo_config_t* c, int bl, int s,
   mg->quota_gap = INFINITY;
   mg->n_commit = 0;
   mg->fired = 0;
+  mg->edit_margin = INFINITY;
+  mg->n_edit = 0;
+  mg->pad = 0;
 
   /* 1. stability */
   int all_eq = s >= 1;
@@ -318,6 +325,19 @@ void ebo_canvas_decide(const ebo_config_t* c, int bl, int s,
     int n = 0;
     for (int l = 0; l < L; ++l)
       if (!committed[l]) open[n++] = l;
+
+    /* BR editing of positions committed before this step */
+    if (c->rule == EBO_RULE_BR && c->editing_threshold >= 0.0) {
+      for (int l = 0; l < L; ++l) {
+        if (!committed[l] || amax[l] == canvas[l]) continue;
+        double d = fabs(pmax[l] - c->editing_threshold);
+        if (d < mg->edit_margin) mg->edit_margin = d;
+        if (pmax[l] >= c->editing_threshold) {
+          canvas[l] = amax[l];
+          mg->n_edit++;
+        }
+      }
+    }
 
     int32_t* pick = (int32_t*)malloc(sizeof(int32_t) * (size_t)(L > 0 ? L : 1));
     int np = 0;

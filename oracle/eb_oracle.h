@@ -83,6 +83,8 @@ typedef struct {
   int32_t group_size;         /* elements per Gumbel group (64 in the library) */
   int32_t canvas_offset;      /* global index of local canvas 0 */
   uint64_t seed;
+  double editing_threshold;   /* BR: re-edit a committed token when the argmax
+                                 differs and pmax >= this; < 0 disables */
 } ebo_config_t;
 
 /* Per-canvas decision margins: how far each decision was from flipping. */
@@ -95,6 +97,10 @@ typedef struct {
   double mean_H;       /* canvas mean entropy (all positions) */
   int32_t n_commit;    /* positions committed this step */
   int32_t fired;       /* 1 if the adaptive stop fired */
+  double edit_margin;  /* BR editing: min |pmax - editing_threshold| over committed
+                          positions whose argmax differs from their token */
+  int32_t n_edit;      /* committed positions re-edited this step */
+  int32_t pad;
 } ebo_margins_t;
 
 void     ebo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);

@@ -86,6 +86,7 @@ class Workload:
     stability_steps: int = 1
     t_max: float = 0.8
     t_min: float = 0.4
+    editing_threshold: float = -1.0
 
     @property
     def elt(self) -> int:
@@ -107,7 +108,7 @@ class Workload:
                     entropy_bound=self.entropy_bound, stop_entropy=self.stop_entropy,
                     stability_steps=self.stability_steps, rule=self.rule,
                     threshold=self.threshold, quota=self.quota, greedy=self.greedy,
-                    seed=self.seed)
+                    seed=self.seed, editing_threshold=self.editing_threshold)
 
     def replace(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

@@ -14,6 +14,8 @@ except where the oracle's own margins say the decision hinges on rounding):
                    the stop threshold
   BR (N5)          excused when a pmax is within 1e-6 of the threshold or the
                    two pmax values at the quota cut differ by <= 1e-5 relative
+  BR edit (N6)     excused when a moved committed position's pmax is within
+                   1e-6 of editing_threshold
 
 CUT_WINDOW and STOP_WINDOW bound the GPU's entropy error on low-entropy rows:
 fp32 accumulation of 64-term groups with the group that holds the maximum
@@ -60,6 +62,8 @@ def canvas_flags(mg: dict) -> list:
         f.append("N4")
     if mg["br_margin"] <= BR_WINDOW or mg["quota_gap"] <= QUOTA_WINDOW:
         f.append("N5")
+    if mg["edit_margin"] <= BR_WINDOW:
+        f.append("N6")
     return f
 
 
@@ -68,6 +72,7 @@ class Stats:
         self.max_dH = 0.0
         self.max_dH_low = 0.0  # positions with H < 0.2 (the ones decisions use)
         self.max_rel_dpmax = 0.0
+        self.edits = 0  # committed positions the oracle re-edited (block refinement)
         self.rows = 0
         self.draws = 0
         self.excused_draws = 0

@@ -46,6 +46,7 @@ def test_default_config_matches_model_card(E):
     assert (c.t_max, c.t_min, c.entropy_bound, c.stop_entropy) == (0.8, 0.4, 0.1, 0.005)
     assert c.stability_steps == 1 and c.rule == E.RULE_ENTROPY_BOUND and c.quota == 6
     assert c.threshold == 0.9 and c.greedy == 0
+    assert c.editing_threshold == -1.0  # block refinement editing off
 
 
 def test_strerror_and_version(E):
@@ -60,7 +61,7 @@ def test_strerror_and_version(E):
     ("L", 0, 1), ("B", 0, 1), ("V", 0, 1), ("num_steps", 0, 1), ("L", 5000, 6),
     ("B", 5000, 6), ("rule", 7, 1), ("greedy", 2, 1), ("t_max", -0.5, 1),
     ("entropy_bound", -1.0, 1), ("stability_steps", -1, 1), ("quota", -2, 1),
-    ("canvas_offset", (1 << 24), 6),
+    ("canvas_offset", (1 << 24), 6), ("editing_threshold", float("nan"), 1),
 ])
 def test_init_validates_config_on_host(E, field, value, code):
     lib = E.library()

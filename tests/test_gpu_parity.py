@@ -90,6 +90,7 @@ def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=3, mask=None):
             out = O.step_canvas(st, i, lg[i], s)
             compare_rows(stats, i, s, Hg[i], amg[i], pmg[i], smg[i], out, range(w.L), f32,
                          out["open_before"])
+            stats.edits += int(out["margins"]["n_edit"])
             differ = bool(np.any((smg[i] != out["sample"]) & out["open_before"]))
             compare_canvas(stats, st, i, s, (cvg[i], cmg[i], spg[i]), out["margins"], differ)
             if st.stop[i]:
@@ -115,6 +116,11 @@ MID = synth.WORKLOADS["canvas"].replace(name="mid", B=3, L=64, V=8232, num_steps
     ("mid_f32_eb", MID.replace(dtype=synth.F32, seed=7)),
     ("mid_bf16_mi", MID.replace(rule=O.RULE_EB_MI, seed=8)),
     ("mid_bf16_br_greedy", MID.replace(rule=O.RULE_BR, greedy=1, quota=3, seed=9)),
+    ("mid_bf16_br_editing", MID.replace(rule=O.RULE_BR, greedy=1, quota=3, seed=14,
+                                        editing_threshold=0.5)),
+    ("mid_f32_br_sampled_editing", MID.replace(dtype=synth.F32, rule=O.RULE_BR, quota=2,
+                                               seed=15, t_max=1.0, t_min=1.0,
+                                               editing_threshold=0.3)),
     ("mid_f32_br_sampled", MID.replace(dtype=synth.F32, rule=O.RULE_BR, quota=2, seed=10,
                                        t_max=1.0, t_min=1.0)),
     ("mid_zipf_f32", MID.replace(kind=synth.ZIPF, dtype=synth.F32, seed=11, B=2)),
@@ -123,7 +129,9 @@ MID = synth.WORKLOADS["canvas"].replace(name="mid", B=3, L=64, V=8232, num_steps
 ])
 def test_full_parity(E, name, w):
     stats = run_full(E, w)
-    print(name, stats)
+    print(name, stats, "edits", stats.edits)
+    if w.editing_threshold >= 0.0:
+        assert stats.edits > 0, "the editing configuration re-edits some committed token"
 
 
 def _mask_neg_inf(V):

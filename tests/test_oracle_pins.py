@@ -330,6 +330,57 @@ def test_br_commit_threshold_plus_quota(oracle_lib):
         assert got == over | set(rest[:q])
 
 
+def test_br_editing_threshold_reedits_confident_committed_positions(oracle_lib):
+    """BlockRefinement with editing (diffusers "DiffusionGemma", Schedulers:
+    editing_threshold lets the scheduler re-edit committed tokens), as read
+    here: a position committed before the step whose argmax differs from its
+    token takes the argmax iff its pmax >= editing_threshold; it stays
+    committed; open positions follow the ordinary rule."""
+    L = 6
+    cfg = O.Config(B=1, L=L, V=1000, rule=O.RULE_BR, stop_entropy=-1.0, threshold=0.9,
+                   quota=1, greedy=1, editing_threshold=0.6)
+    st = O.State(cfg).init()
+    st.committed[0, :4] = 1
+    st.canvas[0, :4] = [10, 11, 12, 13]
+    amax = np.array([20, 21, 12, 23, 24, 25], np.int32)
+    pmax = np.array([0.61, 0.59, 0.99, 0.6, 0.2, 0.1])
+    H = np.full(L, 0.5)
+    mg = O.canvas_decide(st, 0, 3, H, amax, pmax, np.zeros(L, np.int32))
+    # 0: differs, confident -> edited; 1: below the threshold -> kept;
+    # 2: argmax equals the token -> untouched; 3: pmax == threshold -> edited
+    assert st.canvas[0, :4].tolist() == [20, 11, 12, 23]
+    assert st.committed[0, :4].all()
+    assert mg["n_edit"] == 2
+    assert abs(mg["edit_margin"] - 0.0) < 1e-12  # position 3 sits on the threshold
+    # the open positions: quota 1 commits the higher pmax (position 4)
+    assert st.committed[0, 4] == 1 and st.canvas[0, 4] == 24 and st.committed[0, 5] == 0
+    # disabled (negative) or under another rule: no edits
+    for rule, eps in ((O.RULE_BR, -1.0), (O.RULE_EB, 0.6)):
+        cfg2 = O.Config(B=1, L=L, V=1000, rule=rule, stop_entropy=-1.0, greedy=1,
+                        editing_threshold=eps)
+        st2 = O.State(cfg2).init()
+        st2.committed[0, :4] = 1
+        st2.canvas[0, :4] = [10, 11, 12, 13]
+        mg2 = O.canvas_decide(st2, 0, 3, H, amax, pmax, np.zeros(L, np.int32))
+        assert st2.canvas[0, :4].tolist() == [10, 11, 12, 13] and mg2["n_edit"] == 0
+
+
+def test_br_editing_is_not_applied_when_the_stop_fires(oracle_lib):
+    L = 3
+    cfg = O.Config(B=1, L=L, V=1000, rule=O.RULE_BR, stop_entropy=0.5, stability_steps=1,
+                   greedy=1, editing_threshold=0.1)
+    st = O.State(cfg).init()
+    st.committed[0, 0] = 1
+    st.canvas[0, 0] = 10
+    st.prev[0] = [20, 21, 22]
+    st.stable[0] = 0
+    H = np.full(L, 0.01)  # mean below the stop entropy, argmax unchanged
+    mg = O.canvas_decide(st, 0, 4, H, np.array([20, 21, 22], np.int32), np.full(L, 0.99),
+                         np.zeros(L, np.int32))
+    assert mg["fired"] == 1 and mg["n_edit"] == 0
+    assert st.canvas[0].tolist() == [10, 21, 22]  # frozen token kept, open ones take the argmax
+
+
 def test_commit_takes_sample_or_argmax_when_greedy(oracle_lib):
     H = np.array([0.01, 0.5, 0.02, 0.9])
     st, mg, before, smp = _decide_all_open(O.RULE_EB, H)
