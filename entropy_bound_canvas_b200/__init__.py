@@ -52,7 +52,7 @@ class Config(C.Structure):
         ("stability_steps", C.c_int32), ("rule", C.c_int32),
         ("threshold", C.c_double), ("quota", C.c_int32), ("greedy", C.c_int32),
         ("canvas_offset", C.c_int32), ("seed", C.c_uint64),
-        ("editing_threshold", C.c_double),
+        ("editing_threshold", C.c_double), ("vocab_offset", C.c_int32), ("vocab_total", C.c_int32),
     ]
 
 
@@ -84,6 +84,12 @@ def _lib():
         L.eb_sampler_draws.restype = i32
         L.eb_sampler_set_state.argtypes = [vp, vp, vp, i32, vp]
         L.eb_sampler_set_state.restype = i32
+        L.eb_sampler_step_slice.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp]
+        L.eb_sampler_step_slice.restype = i32
+        L.eb_sampler_combine.argtypes = [vp, vp, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.eb_sampler_combine.restype = i32
+        L.eb_slice_record_bytes.argtypes = []
+        L.eb_slice_record_bytes.restype = C.c_size_t
         L.eb_sampler_set_split_event.argtypes = [vp, vp]
         L.eb_sampler_set_split_event.restype = i32
         L.eb_sampler_workspace_bytes.argtypes = [vp]
@@ -213,6 +219,75 @@ class EBSampler:
             self._ptr(argmax, torch.int32, (self.B, self.L), "argmax"),
             self._ptr(stop_flags, torch.uint8, (self.B,), "stop_flags"), self._stream()),
             "eb_sampler_step")
+
+    # -- vocabulary-sharded logits ---------------------------------------------
+    def slice_records(self):
+        """A records buffer for one slice: [B, L, record bytes] uint8."""
+        torch = _torch()
+        n = int(_lib().eb_slice_record_bytes())
+        return torch.empty((self.B, self.L, n), dtype=torch.uint8, device=self.device)
+
+    def step_slice(self, logits, step: int, committed, stop_flags, records):
+        """This device's vocabulary slice of a step: per-position records."""
+        torch = _torch()
+        dt = self._dtype(logits)
+        n = int(_lib().eb_slice_record_bytes())
+        _check(_lib().eb_sampler_step_slice(
+            self._h, C.c_void_p(logits.data_ptr()), dt, int(step),
+            self._ptr(committed, torch.uint8, (self.B, self.L), "committed"),
+            self._ptr(stop_flags, torch.uint8, (self.B,), "stop_flags"),
+            self._ptr(records, torch.uint8, (self.B, self.L, n), "records"), self._stream()),
+            "eb_sampler_step_slice")
+
+    def combine(self, all_records, step: int, canvas, committed, entropies, argmax, stop_flags):
+        """Every slice's records ([n_slices, B, L, record bytes], slice order) ->
+        the step's results and canvas decisions, as step() gives them."""
+        torch = _torch()
+        n = int(_lib().eb_slice_record_bytes())
+        if all_records.dim() != 4 or tuple(all_records.shape[1:]) != (self.B, self.L, n):
+            raise ValueError(f"records must be [n_slices, {self.B}, {self.L}, {n}]")
+        _check(_lib().eb_sampler_combine(
+            self._h, self._ptr(all_records, torch.uint8, None, "records"),
+            int(all_records.shape[0]), int(step),
+            self._ptr(canvas, torch.int32, (self.B, self.L), "canvas"),
+            self._ptr(committed, torch.uint8, (self.B, self.L), "committed"),
+            self._ptr(entropies, torch.float32, (self.B, self.L), "entropies"),
+            self._ptr(argmax, torch.int32, (self.B, self.L), "argmax"),
+            self._ptr(stop_flags, torch.uint8, (self.B,), "stop_flags"), self._stream()),
+            "eb_sampler_combine")
+
+    def step_split(self, logits, step: int, canvas, committed, entropies, argmax, stop_flags,
+                   group=None):
+        """A step over vocabulary-sharded logits: this rank's slice, one
+        all-gather of the records over `group` (ranks ordered by slice), then
+        the combine.  Without a process group the handle is the only slice."""
+        torch = _torch()
+        rec = self.slice_records()
+        self.step_slice(logits, step, committed, stop_flags, rec)
+        world = 1
+        if group is not None or (torch.distributed.is_available()
+                                 and torch.distributed.is_initialized()):
+            world = torch.distributed.get_world_size(group)
+        if world == 1:
+            allr = rec.unsqueeze(0)
+        else:
+            allr = torch.empty((world,) + tuple(rec.shape), dtype=rec.dtype, device=rec.device)
+            torch.distributed.all_gather_into_tensor(allr, rec, group=group)
+        self.combine(allr, step, canvas, committed, entropies, argmax, stop_flags)
+
+    def _dtype(self, logits):
+        torch = _torch()
+        if logits.dtype == torch.float32:
+            dt = F32
+        elif logits.dtype == torch.bfloat16:
+            dt = BF16
+        else:
+            raise TypeError("logits must be float32 or bfloat16")
+        if logits.device != self.device or tuple(logits.shape) != (self.B, self.L, self.V):
+            raise ValueError(f"logits must be [{self.B}, {self.L}, {self.V}] on {self.device}")
+        if not logits.is_contiguous():
+            raise ValueError("logits must be contiguous")
+        return dt
 
     def step_ptr(self, logits_ptr: int, dtype: int, step: int, canvas_ptr: int,
                  committed_ptr: int, entropies_ptr: int, argmax_ptr: int, stop_ptr: int,

@@ -40,6 +40,19 @@ struct Partial {
   int gidx;
 };
 
+// What one vocabulary slice contributes to a position (vocabulary-sharded
+// logits): sums relative to the slice maximum (d = (z - zmax) c2, log2
+// units), its argmax and its part of the draw, with global ids.  40 bytes.
+struct SliceRecord {
+  double S, W;
+  float zmax;
+  float gscore;  // best group score of the slice (-inf: none)
+  int32_t amax;
+  int32_t sample;  // element drawn in the slice's best group (-1: none)
+  int32_t pad0, pad1;
+};
+static_assert(sizeof(SliceRecord) == 40, "slice record layout");
+
 struct StepArgs {
   const void* logits;
   int32_t* canvas;
@@ -65,6 +78,8 @@ struct StepArgs {
   float c2, iT;
   double gamma, tau, theta;
   double eps_edit;  // block refinement editing threshold; < 0: no editing
+  int v_off;        // global id of local logit 0 (vocabulary slice; a multiple of 64)
+  int V_tot;        // global vocabulary size (renoise range, token check)
   uint32_t key0, key1;
 };
 

@@ -136,7 +136,11 @@ __device__ __forceinline__ unsigned long long key_desc(float p, int l) {
 // ---------------------------------------------------------------------------
 struct RowOut {
   float H, pmax;
-  int amax, sample;
+  int amax, sample;  // global vocabulary ids
+  // the same sums before the entropy, for a vocabulary slice's record:
+  // S = sum 2^d, W = sum 2^d d, d = (z - zmax) c2, and the best group score
+  double S, W;
+  float zmax, gscore;
 };
 
 // The PER logits v0 .. v0 + PER - 1 of one row (those >= V read as -inf):
@@ -235,7 +239,8 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
   if (draw) {
 #pragma unroll
     for (int c = 0; c < NC; ++c) {
-      const Words4 w = philox(((uint32_t)vs0 >> 2) + (uint32_t)c, (uint32_t)l, (uint32_t)a.s, c3,
+      const Words4 w = philox(((uint32_t)(a.v_off + vs0) >> 2) + (uint32_t)c, (uint32_t)l,
+                              (uint32_t)a.s, c3,
                               a.key0, a.key1);
 #pragma unroll
       for (int q = 0; q < 4; ++q) xw[4 * c + q] = w.w[q];
@@ -273,14 +278,18 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
   const double W = (double)wsum + (double)R.Wrest;
   out.H = (float)(log(S) - 0.6931471805599453 * (W / S));
   out.pmax = (float)(1.0 / S);
-  out.amax = am;
+  out.amax = am == 0x7fffffff ? am : am + a.v_off;
+  out.S = S;
+  out.W = W;
+  out.zmax = R.zmax;
+  out.gscore = R.gscore;
   if (valid && (!isfinite(S) || !isfinite(W) || am == 0x7fffffff))
     atomicOr(a.status, kStatusNonFinite);
 
   // 4. the categorical draw within the winning group: the largest tempered
   //    logit is drawn first; the logarithms of every element that cannot
   //    beat it are skipped exactly
-  out.sample = open ? am : -1;
+  out.sample = open ? out.amax : -1;
   if (__any_sync(0xffffffffu, draw)) {
     float ymax = -INFINITY;
     int emax = -1;
@@ -350,7 +359,7 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
         barg = oa;
       }
     }
-    if (draw) out.sample = barg;
+    if (draw) out.sample = barg == 0x7fffffff ? barg : barg + a.v_off;
   }
   return out;
 }
@@ -418,7 +427,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
     if (a.s >= 1 && sAm[l] != sPrev[l]) neq = 1;
     if (!sOpen[l]) {
       const int tok = sTok[l];
-      if (tok < 0 || tok >= a.V) atomicOr(a.status, kStatusBadToken);
+      if (tok < 0 || tok >= a.V_tot) atomicOr(a.status, kStatusBadToken);
     } else if (!br) {
       ncand += (double)sH[l] <= a.gamma ? 1 : 0;
     } else if (!((double)sPm[l] >= a.theta)) {
@@ -503,7 +512,8 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
         ++left;
         const Words4 r = philox((uint32_t)l >> 2, 0u, (uint32_t)a.s, bg | (kStreamRenoise << 24),
                                 a.key0, a.key1);
-        a.canvas[row0 + l] = (int32_t)uniform_token(pick_word(r, (uint32_t)l & 3u), (uint32_t)a.V);
+        a.canvas[row0 + l] =
+            (int32_t)uniform_token(pick_word(r, (uint32_t)l & 3u), (uint32_t)a.V_tot);
       }
     }
     a.prev_amax[row0 + l] = sAm[l];
@@ -586,6 +596,127 @@ __global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThread
     case 8: finish_rows<DT, 8>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
     case 16: finish_rows<DT, 16>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
     default: finish_rows<DT, 32>(a, lay, smem, cluster, bi, ai, rank, open, NG); break;
+  }
+  cluster.sync();  // rank 0 now holds every position's results
+  if (rank == 0)
+    canvas_epilogue(a, bi, ctrl, reinterpret_cast<const float*>(smem + lay.H),
+                    reinterpret_cast<const int*>(smem + lay.am),
+                    reinterpret_cast<const int*>(smem + lay.smp),
+                    reinterpret_cast<const float*>(smem + lay.pm),
+                    reinterpret_cast<const int*>(smem + lay.prev),
+                    reinterpret_cast<const int*>(smem + lay.tok), smem + lay.open,
+                    smem + lay.pick, reinterpret_cast<unsigned long long*>(smem + lay.keys));
+}
+
+// ---------------------------------------------------------------------------
+// Vocabulary-sharded logits
+// ---------------------------------------------------------------------------
+// Slice records: after the stream kernel ran over this device's slice, every
+// position of an active canvas gets its SliceRecord (8-lane subgroups, the
+// same per-position work as the finish kernel, without the epilogue).
+template <int DT>
+__global__ void __launch_bounds__(256) slice_finish_kernel(const StepArgs a,
+                                                           const int32_t* act_index,
+                                                           const int32_t* n_act_ptr,
+                                                           SliceRecord* records) {
+  constexpr int kTPR = 8;
+  const int bi = blockIdx.y;
+  const int tid = threadIdx.x;
+  const int l = blockIdx.x * (256 / kTPR) + tid / kTPR;
+  const int sl = tid % kTPR;
+  const bool in_range = l < a.L;
+  const bool open = in_range && a.committed[(size_t)bi * (size_t)a.L + (size_t)l] == 0;
+  griddep_wait();  // the stream kernel's records and active list are visible
+  const int ai = act_index[bi];
+  if (ai < 0) return;  // uniform over the CTA: a stopped canvas has no records
+  const unsigned long long NG =
+      (unsigned long long)(*n_act_ptr) * (unsigned long long)a.L * (unsigned long long)a.ng;
+  const RowOut ro = finish_row<DT, kTPR>(a, bi, ai, in_range ? l : 0, in_range, open, sl, NG);
+  if (in_range && sl == 0) {
+    SliceRecord r;
+    r.S = ro.S;
+    r.W = ro.W;
+    r.zmax = ro.zmax;
+    r.gscore = ro.gscore;
+    r.amax = ro.amax;
+    r.sample = open && !a.greedy ? ro.sample : -1;
+    r.pad0 = r.pad1 = 0;
+    records[(size_t)bi * (size_t)a.L + (size_t)l] = r;
+  }
+}
+
+// Combine: the n slices' records of each position, in slice order, give the
+// position's entropy, max probability, argmax and draw (the largest slice
+// maximum; the sums rescaled to it; the first slice attaining it for the
+// argmax; the best slice score, earlier slice on a tie, for the draw);
+// then the canvas epilogue, as in finish_kernel.
+template <int DT>
+__global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThreads, 2)
+    combine_kernel(const StepArgs a, const int32_t* act_index, const SliceRecord* records,
+                   int n_slices) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  const FinLayout lay = fin_layout(a.L);
+  FinCtrl* ctrl = reinterpret_cast<FinCtrl*>(smem + lay.ctrl);
+  cgr::cluster_group cluster = cgr::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int bi = blockIdx.x / kFinCluster;
+  const int tid = threadIdx.x;
+  const int rpc = fin_rows_per_cta(a.L);
+  if (act_index[bi] < 0) return;  // uniform over the cluster: a stopped canvas is untouched
+  if (rank == 0) {
+    const size_t row0 = (size_t)bi * (size_t)a.L;
+    int* sPrev = reinterpret_cast<int*>(smem + lay.prev);
+    int* sTok = reinterpret_cast<int*>(smem + lay.tok);
+    for (int i = tid; i < a.L; i += kFinThreads) {
+      sPrev[i] = a.prev_amax[row0 + i];
+      sTok[i] = a.canvas[row0 + i];
+    }
+    if (tid == 0) ctrl->stable_prev = a.stable[bi];
+  }
+  cluster.sync();  // every CTA of the cluster runs: its shared memory may be written
+  for (int k = tid; k < rpc; k += kFinThreads) {
+    const int l = rank * rpc + k;
+    if (l >= a.L) break;
+    const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
+    const size_t stride = (size_t)a.B * (size_t)a.L;
+    float M = -INFINITY;
+    int am = 0x7fffffff;
+    for (int g = 0; g < n_slices; ++g) {
+      const SliceRecord& r = records[(size_t)g * stride + grow];
+      if (r.zmax > M) {
+        M = r.zmax;
+        am = r.amax;
+      }
+    }
+    double S = 0.0, W = 0.0;
+    float best = -INFINITY;
+    int x = -1;
+    for (int g = 0; g < n_slices; ++g) {
+      const SliceRecord r = records[(size_t)g * stride + grow];
+      if (r.gscore > best) {
+        best = r.gscore;
+        x = r.sample;
+      }
+      if (!(r.zmax > -INFINITY)) continue;
+      const double dd = (double)(r.zmax - M) * (double)a.c2;
+      const double f = exp2(dd);
+      S += f * r.S;
+      W += f * (r.W + dd * r.S);
+    }
+    const float H = (float)(log(S) - 0.6931471805599453 * (W / S));
+    const float pm = (float)(1.0 / S);
+    if (!isfinite(S) || !isfinite(W) || am == 0x7fffffff) atomicOr(a.status, kStatusNonFinite);
+    const bool open = a.committed[grow] == 0;
+    const int smp = open ? (a.greedy || x < 0 ? am : x) : -1;
+    a.H_out[grow] = H;
+    a.amax_out[grow] = am;
+    a.sample[grow] = smp;
+    a.pmax[grow] = pm;
+    *cluster.map_shared_rank(reinterpret_cast<float*>(smem + lay.H) + l, 0) = H;
+    *cluster.map_shared_rank(reinterpret_cast<int*>(smem + lay.am) + l, 0) = am;
+    *cluster.map_shared_rank(reinterpret_cast<int*>(smem + lay.smp) + l, 0) = smp;
+    *cluster.map_shared_rank(reinterpret_cast<float*>(smem + lay.pm) + l, 0) = pm;
+    *cluster.map_shared_rank(smem + lay.open + l, 0) = open ? 1 : 0;
   }
   cluster.sync();  // rank 0 now holds every position's results
   if (rank == 0)

@@ -43,6 +43,9 @@ struct eb_sampler {
   int nw = 0;        // records per (row, stream CTA)
   KernelCfg k[2];     // stream kernel [dtype]
   KernelCfg fin[2];   // finish kernel [dtype]
+  KernelCfg combine;  // combine kernel (vocabulary slices)
+  int V_tot = 0;      // global vocabulary size
+  int slice_step = -1;
   // workspace (one allocation)
   void* ws = nullptr;
   size_t ws_bytes = 0;
@@ -91,6 +94,12 @@ int validate_config(const eb_config_t* c) {
   if (std::isnan(c->stop_entropy) || std::isnan(c->threshold) || std::isnan(c->editing_threshold))
     return EB_ERR_INVALID_ARG;
   if (c->stability_steps < 0 || c->quota < 0) return EB_ERR_INVALID_ARG;
+  // a vocabulary slice starts on a group boundary and lies inside the vocabulary
+  if (c->vocab_offset < 0 || c->vocab_offset % ebk::kGroup != 0 || c->vocab_total < 0)
+    return EB_ERR_INVALID_ARG;
+  if (c->vocab_total > 0 && (int64_t)c->vocab_offset + c->V > (int64_t)c->vocab_total)
+    return EB_ERR_INVALID_ARG;
+  if (c->vocab_total == 0 && c->vocab_offset != 0) return EB_ERR_INVALID_ARG;
   // group numbering fits the 64-bit work split: B * L * ng * grid < 2^63
   const uint64_t ng = ((uint64_t)c->V + ebk::kGroup - 1) / ebk::kGroup;
   if ((uint64_t)c->B * (uint64_t)c->L * ng >= (1ull << 46)) return EB_ERR_OVERFLOW;
@@ -134,6 +143,18 @@ int setup_finish(eb_sampler* h, const cudaDeviceProp& prop) {
   return EB_OK;
 }
 
+int setup_combine(eb_sampler* h, const cudaDeviceProp& prop) {
+  KernelCfg& kc = h->combine;
+  kc.fn = reinterpret_cast<const void*>(&ebk::combine_kernel<ebk::kBF16>);
+  kc.smem = ebk::fin_layout(h->cfg.L).total;
+  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
+  if (cudaFuncSetAttribute(ebk::combine_kernel<ebk::kBF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kc.smem) != cudaSuccess)
+    return EB_ERR_CUDA;
+  kc.grid = h->cfg.B * ebk::kFinCluster;
+  return EB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -157,6 +178,8 @@ void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V) {
   cfg->canvas_offset = 0;
   cfg->seed = 0;
   cfg->editing_threshold = -1.0;
+  cfg->vocab_offset = 0;
+  cfg->vocab_total = 0;
 }
 
 int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
@@ -183,10 +206,11 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   if ((rc = setup_kernel<ebk::kF32>(h, prop)) != EB_OK ||
       (rc = setup_kernel<ebk::kBF16>(h, prop)) != EB_OK ||
       (rc = setup_finish<ebk::kF32>(h, prop)) != EB_OK ||
-      (rc = setup_finish<ebk::kBF16>(h, prop)) != EB_OK) {
+      (rc = setup_finish<ebk::kBF16>(h, prop)) != EB_OK || (rc = setup_combine(h, prop)) != EB_OK) {
     delete h;
     return rc;
   }
+  h->V_tot = cfg->vocab_total > 0 ? cfg->vocab_total : cfg->V;
   // Most CTAs one row can span: with one active canvas each CTA owns at
   // least floor(L ng / G) groups, so a row meets at most
   // floor((ng - 1) G / (L ng)) + 2 of them.
@@ -244,39 +268,32 @@ int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
   if (!guard.ok) return EB_ERR_CUDA;
   const eb_config_t& c = h->cfg;
   ebk::init_canvas_kernel<<<c.B, 256, 0, (cudaStream_t)stream>>>(
-      canvas, committed, stop_flags, h->stable, c.L, c.V, c.canvas_offset,
+      canvas, committed, stop_flags, h->stable, c.L, h->V_tot, c.canvas_offset,
       (uint32_t)(c.seed & 0xffffffffu), (uint32_t)(c.seed >> 32));
   if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = -1;
+  h->slice_step = -1;
   return EB_OK;
 }
 
-int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, int32_t* canvas,
-                    uint8_t* committed, float* entropies, int32_t* argmax, uint8_t* stop_flags,
-                    void* stream) {
-  if (!h || !logits || !canvas || !committed || !entropies || !argmax || !stop_flags)
-    return EB_ERR_INVALID_ARG;
-  if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
-  if ((uintptr_t)logits % (dtype == EB_F32 ? 4u : 2u) != 0) return EB_ERR_INVALID_ARG;
-  const eb_config_t& c = h->cfg;
-  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
-  if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
-  DeviceGuard guard(h->device);
-  if (!guard.ok) return EB_ERR_CUDA;
-  cudaStream_t st = (cudaStream_t)stream;
+}  // extern "C"
 
-  const double T = c.greedy ? 1.0
-                   : c.num_steps <= 1
-                       ? c.t_max
-                       : c.t_max + (c.t_min - c.t_max) * (double)step / (double)(c.num_steps - 1);
-  StepArgs a;
+namespace {
+
+// Temperature of step s: linear from t_max to t_min over num_steps (T = 1
+// when greedy).
+double step_temperature(const eb_config_t& c, int step) {
+  return c.greedy ? 1.0
+         : c.num_steps <= 1
+             ? c.t_max
+             : c.t_max + (c.t_min - c.t_max) * (double)step / (double)(c.num_steps - 1);
+}
+
+// The step's arguments that do not depend on the caller's buffers.
+void fill_args(const eb_sampler* h, StepArgs& a, int step) {
+  const eb_config_t& c = h->cfg;
+  const double T = step_temperature(c, step);
   std::memset(&a, 0, sizeof(a));
-  a.logits = logits;
-  a.canvas = canvas;
-  a.committed = committed;
-  a.H_out = entropies;
-  a.amax_out = argmax;
-  a.stop_flags = stop_flags;
   a.partials = h->partials;
   a.prev_amax = h->prev_amax;
   a.stable = h->stable;
@@ -305,18 +322,75 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.tau = c.stop_entropy;
   a.theta = c.threshold;
   a.eps_edit = c.rule == EB_RULE_BLOCK_REFINEMENT ? c.editing_threshold : -1.0;
+  a.v_off = c.vocab_offset;
+  a.V_tot = h->V_tot;
   a.key0 = (uint32_t)(c.seed & 0xffffffffu);
   a.key1 = (uint32_t)(c.seed >> 32);
+}
 
+// The stream kernel over `logits` (this device's rows or vocabulary slice).
+int launch_stream(eb_sampler* h, StepArgs& a, const void* logits, int dtype, cudaStream_t st) {
   const size_t elt = dtype == EB_F32 ? 4 : 2;
-  const bool vec = ((uintptr_t)logits % 16 == 0) && (((size_t)c.V * elt) % 16 == 0);
+  a.logits = logits;
+  a.vec_ok = ((uintptr_t)logits % 16 == 0) && (((size_t)h->cfg.V * elt) % 16 == 0) ? 1 : 0;
   const KernelCfg& kc = h->k[dtype];
   a.G1 = kc.grid;
-  a.vec_ok = vec ? 1 : 0;
   void* args[] = {&a};
   if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), args, kc.smem, st) !=
       cudaSuccess)
     return EB_ERR_CUDA;
+  return EB_OK;
+}
+
+// A kernel launched as a programmatic dependent of the previous one on `st`.
+int launch_dependent(const void* fn, dim3 grid, dim3 block, size_t smem, void** args,
+                     cudaStream_t st) {
+  cudaLaunchConfig_t lc;
+  std::memset(&lc, 0, sizeof(lc));
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = attr;
+  lc.numAttrs = 1;
+  return cudaLaunchKernelExC(&lc, fn, args) == cudaSuccess ? EB_OK : EB_ERR_CUDA;
+}
+
+bool is_slice(const eb_sampler* h) {
+  return h->cfg.vocab_offset != 0 || h->V_tot != h->cfg.V;
+}
+
+}  // namespace
+
+extern "C" {
+
+int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, int32_t* canvas,
+                    uint8_t* committed, float* entropies, int32_t* argmax, uint8_t* stop_flags,
+                    void* stream) {
+  if (!h || !logits || !canvas || !committed || !entropies || !argmax || !stop_flags)
+    return EB_ERR_INVALID_ARG;
+  if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
+  if ((uintptr_t)logits % (dtype == EB_F32 ? 4u : 2u) != 0) return EB_ERR_INVALID_ARG;
+  if (is_slice(h)) return EB_ERR_INVALID_ARG;  // a vocabulary slice steps by slice + combine
+  const eb_config_t& c = h->cfg;
+  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
+  if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  StepArgs a;
+  fill_args(h, a, step);
+  a.canvas = canvas;
+  a.committed = committed;
+  a.H_out = entropies;
+  a.amax_out = argmax;
+  a.stop_flags = stop_flags;
+  int rc = launch_stream(h, a, logits, dtype, st);
+  if (rc != EB_OK) return rc;
 
   if (h->split_event && cudaEventRecord(h->split_event, st) != cudaSuccess) return EB_ERR_CUDA;
 
@@ -324,21 +398,77 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   const int32_t* act_index = h->act_index;
   const int32_t* n_act = h->n_act;
   void* fargs[] = {&a, &act_index, &n_act};
-  cudaLaunchConfig_t lc;
-  std::memset(&lc, 0, sizeof(lc));
-  lc.gridDim = dim3(kf.grid);
-  lc.blockDim = dim3(ebk::kFinThreads);
-  lc.dynamicSmemBytes = kf.smem;
-  lc.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  lc.attrs = attr;
-  lc.numAttrs = 1;
-  if (cudaLaunchKernelExC(&lc, kf.fn, fargs) != cudaSuccess) return EB_ERR_CUDA;
+  rc = launch_dependent(kf.fn, dim3(kf.grid), dim3(ebk::kFinThreads), kf.smem, fargs, st);
+  if (rc != EB_OK) return rc;
   h->last_step = step;
   return EB_OK;
 }
+
+int eb_sampler_step_slice(eb_sampler_t* h, const void* logits, int dtype, int step,
+                          const uint8_t* committed, const uint8_t* stop_flags, void* records,
+                          void* stream) {
+  if (!h || !logits || !committed || !stop_flags || !records) return EB_ERR_INVALID_ARG;
+  if (dtype != EB_F32 && dtype != EB_BF16) return EB_ERR_UNSUPPORTED;
+  if ((uintptr_t)logits % (dtype == EB_F32 ? 4u : 2u) != 0 || (uintptr_t)records % 8 != 0)
+    return EB_ERR_INVALID_ARG;
+  const eb_config_t& c = h->cfg;
+  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
+  if (step != 0 && step != h->slice_step + 1) return EB_ERR_STEP_ORDER;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  StepArgs a;
+  fill_args(h, a, step);
+  a.committed = const_cast<uint8_t*>(committed);  // read only on this path
+  a.stop_flags = const_cast<uint8_t*>(stop_flags);
+  int rc = launch_stream(h, a, logits, dtype, st);
+  if (rc != EB_OK) return rc;
+  const int32_t* act_index = h->act_index;
+  const int32_t* n_act = h->n_act;
+  ebk::SliceRecord* rec = static_cast<ebk::SliceRecord*>(records);
+  void* sargs[] = {&a, &act_index, &n_act, &rec};
+  const void* fn = dtype == EB_F32 ? reinterpret_cast<const void*>(&ebk::slice_finish_kernel<ebk::kF32>)
+                                   : reinterpret_cast<const void*>(&ebk::slice_finish_kernel<ebk::kBF16>);
+  rc = launch_dependent(fn, dim3((unsigned)((c.L + 31) / 32), (unsigned)c.B), dim3(256), 0, sargs,
+                        st);
+  if (rc != EB_OK) return rc;
+  h->slice_step = step;
+  return EB_OK;
+}
+
+int eb_sampler_combine(eb_sampler_t* h, const void* records, int n_slices, int step,
+                       int32_t* canvas, uint8_t* committed, float* entropies, int32_t* argmax,
+                       uint8_t* stop_flags, void* stream) {
+  if (!h || !records || !canvas || !committed || !entropies || !argmax || !stop_flags ||
+      n_slices < 1 || (uintptr_t)records % 8 != 0)
+    return EB_ERR_INVALID_ARG;
+  const eb_config_t& c = h->cfg;
+  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
+  if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
+  if (h->slice_step != step) return EB_ERR_STEP_ORDER;  // this handle's slice of the step first
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  StepArgs a;
+  fill_args(h, a, step);
+  a.canvas = canvas;
+  a.committed = committed;
+  a.H_out = entropies;
+  a.amax_out = argmax;
+  a.stop_flags = stop_flags;
+  const int32_t* act_index = h->act_index;
+  const ebk::SliceRecord* rec = static_cast<const ebk::SliceRecord*>(records);
+  void* cargs[] = {&a, &act_index, &rec, &n_slices};
+  if (cudaLaunchKernel(h->combine.fn, dim3(h->combine.grid), dim3(ebk::kFinThreads), cargs,
+                       h->combine.smem, st) != cudaSuccess)
+    return EB_ERR_CUDA;
+  h->last_step = step;
+  return EB_OK;
+}
+
+size_t eb_slice_record_bytes(void) { return sizeof(ebk::SliceRecord); }
 
 int eb_canvas_done(eb_sampler_t* h, const uint8_t* stop_flags, int b, int* done, void* stream) {
   if (!h || !stop_flags || !done) return EB_ERR_INVALID_ARG;
@@ -456,7 +586,7 @@ const char* eb_strerror(int code) {
   }
 }
 
-int eb_version(void) { return 101; }
+int eb_version(void) { return 102; }
 
 }  // extern "C"
 

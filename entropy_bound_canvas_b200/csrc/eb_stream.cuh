@@ -321,13 +321,14 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       const TileMeta m = meta[st];
       if (m.sampling) {
         uint32_t* wd = words + st * Sh::kStageGroups;
-        const int c0 = m.j0 >> 2, c1 = (m.j0 + m.cnt - 1) >> 2;
+        const int gj0 = (a.v_off >> 6) + m.j0;  // global group id of the tile's first group
+        const int c0 = gj0 >> 2, c1 = (gj0 + m.cnt - 1) >> 2;
         const uint32_t c3 = (uint32_t)(a.canvas_offset + m.bi) | (kStreamGroup << 24);
         for (int c = c0 + lane; c <= c1; c += 32) {
           const Words4 w = philox((uint32_t)c, (uint32_t)m.l, (uint32_t)a.s, c3, a.key0, a.key1);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int j = 4 * c + q - m.j0;
+            const int j = 4 * c + q - gj0;
             if (j >= 0 && j < m.cnt) wd[j] = w.w[q];
           }
         }

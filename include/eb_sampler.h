@@ -125,6 +125,10 @@ typedef struct {
                                this step's argmax when the argmax differs from its token
                                and pmax >= editing_threshold; it stays committed.  < 0
                                (the default) disables it; other rules ignore it.  Not NaN. */
+  int32_t vocab_offset;    /* vocabulary-sharded logits: global id of this handle's first
+                              logit, a multiple of EB_GUMBEL_GROUP (0 when not sharded) */
+  int32_t vocab_total;     /* vocabulary-sharded logits: the full vocabulary size, >= 
+                              vocab_offset + V; 0 when not sharded (then V is the vocabulary) */
 } eb_config_t;
 
 /* Fill *cfg with the model card's settings for B canvases of L x V. */
@@ -212,6 +216,39 @@ int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int3
 #define EB_NOALLOC_SCRATCH_BYTES (8u << 20)
 int eb_row_stats_noalloc(const void* logits, int dtype, int32_t rows, int32_t V,
                          double temperature, float* entropies, int32_t* argmax, void* stream);
+
+/* Vocabulary-sharded logits (a tensor-parallel LM head gives each device a
+   contiguous slice of the vocabulary).  Each device's handle is configured
+   with its slice (V = slice width, vocab_offset, vocab_total); all keep the
+   same canvas state.  A step is then three calls, the middle one the
+   caller's collective:
+     1. eb_sampler_step_slice on every device: reads the slice's logits
+        ([B][L][V], dtype as in eb_sampler_step) and writes one
+        eb_slice_record_bytes() record per position ([B][L], device memory,
+        8-byte aligned, caller-owned) -- the slice's maximum, sums, argmax and
+        its part of the two-level draw, with global ids;
+     2. the caller all-gathers the records of every device into one buffer
+        [n_slices][B][L], slices in increasing vocab_offset (rank order of a
+        torch.distributed all_gather_into_tensor with ranks ordered by slice);
+     3. eb_sampler_combine on every device: combines each position's records
+        in slice order (the same arithmetic everywhere, so every device
+        computes the same results) and runs the canvas decisions; outputs as
+        in eb_sampler_step.
+   The results equal eb_sampler_step over the full vocabulary: the maximum,
+   argmax and draw exactly (the draw's groups never straddle slices and
+   every Philox counter uses global ids), the entropies to rounding.
+   eb_sampler_step refuses a slice handle (EB_ERR_INVALID_ARG).  Step order
+   as in eb_sampler_step; eb_sampler_combine needs this handle's
+   eb_sampler_step_slice of the same step first (EB_ERR_STEP_ORDER).  The
+   split follows the pages' model size (one accelerator) only as an
+   extension: no counterpart in the DiffusionGemma pages. */
+int eb_sampler_step_slice(eb_sampler_t* h, const void* logits, int dtype, int step,
+                          const uint8_t* committed, const uint8_t* stop_flags, void* records,
+                          void* stream);
+int eb_sampler_combine(eb_sampler_t* h, const void* records, int n_slices, int step,
+                       int32_t* canvas, uint8_t* committed, float* entropies, int32_t* argmax,
+                       uint8_t* stop_flags, void* stream);
+size_t eb_slice_record_bytes(void);
 
 /* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
    the caller) is non-NULL, every following eb_sampler_step records it on

@@ -128,6 +128,12 @@ def lib():
             L.ebo_row_stats.argtypes = [C.c_void_p, C.c_int, C.c_int, C.c_double,
                                         f64p, f64p, i32p, f64p]
             L.ebo_row_stats.restype = None
+            L.ebo_slice_record.argtypes = [cfgp, C.c_void_p, C.c_int, C.c_int, C.c_int, C.c_double,
+                                           C.c_int, C.c_int, C.c_int, C.POINTER(Slice)]
+            L.ebo_slice_record.restype = None
+            L.ebo_combine_slices.argtypes = [C.POINTER(Slice), C.c_int, C.c_double, f64p, f64p,
+                                             i32p, i32p]
+            L.ebo_combine_slices.restype = None
             L.ebo_sample.argtypes = [cfgp, C.c_void_p, C.c_int, C.c_double, C.c_int, C.c_int,
                                      C.c_int, f64p, i32p]
             L.ebo_sample.restype = C.c_int32
@@ -207,6 +213,31 @@ def sample(cfg: Config, row, inv_T: float, b: int, l: int, s: int):
     mg, gr = C.c_double(), C.c_int32()
     x = lib().ebo_sample(C.byref(c), r.ctypes.data, dt, inv_T, b, l, s, C.byref(mg), C.byref(gr))
     return int(x), mg.value, gr.value
+
+
+class Slice(C.Structure):
+    _fields_ = [("S", C.c_double), ("W", C.c_double), ("zmax", C.c_double),
+                ("gscore", C.c_double), ("amax", C.c_int32), ("sample", C.c_int32)]
+
+
+def slice_record(cfg: Config, row_slice, v_off: int, inv_T: float, b: int, l: int, s: int):
+    """A vocabulary slice's contribution (ebo_slice_t) for one position."""
+    r, dt = _row(row_slice)
+    c = cfg.c()
+    out = Slice()
+    lib().ebo_slice_record(C.byref(c), r.ctypes.data, dt, r.size, v_off, inv_T, b, l, s,
+                           C.byref(out))
+    return out
+
+
+def combine_slices(slices, inv_T: float):
+    """(H, pmax, amax, sample) of a row from its slices in increasing v_off."""
+    arr = (Slice * len(slices))(*slices)
+    H, pm = C.c_double(), C.c_double()
+    am, x = C.c_int32(), C.c_int32()
+    lib().ebo_combine_slices(arr, len(slices), inv_T, C.byref(H), C.byref(pm), C.byref(am),
+                             C.byref(x))
+    return H.value, pm.value, am.value, x.value
 
 
 def sample_flat(cfg: Config, row, inv_T: float, b: int, l: int, s: int):

@@ -210,6 +210,98 @@ int32_t ebo_sample(const ebo_config_t* c, const void* row, int dtype, double inv
 }
 
 /* ------------------------------------------------------------------------- */
+/* Vocabulary-sharded logits                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* One slice [v_off, v_off + V_slice) of a row (v_off a multiple of
+   group_size, so that the draw's groups are whole), with global ids in every
+   Philox counter: the quantities the full-row functions above build from it. */
+void ebo_slice_record(const ebo_config_t* c, const void* row_slice, int dtype, int V_slice,
+                      int v_off, double inv_T, int b, int l, int s, ebo_slice_t* out) {
+  const int G = c->group_size;
+  uint32_t bg = (uint32_t)(c->canvas_offset + b);
+  double zmax = -INFINITY;
+  int32_t am = -1;
+  for (int v = 0; v < V_slice; ++v) {
+    double z = load_z(row_slice, dtype, v);
+    if (z > zmax) { zmax = z; am = v_off + v; }
+  }
+  double m = zmax * inv_T, S = 0.0, W = 0.0;
+  for (int v = 0; v < V_slice; ++v) {
+    double d = load_z(row_slice, dtype, v) * inv_T - m;
+    double e = exp(d);
+    if (e > 0.0) { S += e; W += e * d; }
+  }
+  out->S = S;
+  out->W = W;
+  out->zmax = zmax;
+  out->amax = am;
+  /* two-level draw restricted to the slice's groups (global group ids) */
+  const int ng = (V_slice + G - 1) / G;
+  double best = -INFINITY;
+  int jbest = -1;
+  for (int jl = 0; jl < ng; ++jl) {
+    int lo = jl * G, hi = lo + G < V_slice ? lo + G : V_slice;
+    double mj = -INFINITY;
+    for (int v = lo; v < hi; ++v) {
+      double y = load_z(row_slice, dtype, v) * inv_T;
+      if (y > mj) mj = y;
+    }
+    if (!(mj > -INFINITY)) continue;
+    double Sj = 0.0;
+    for (int v = lo; v < hi; ++v) Sj += exp(load_z(row_slice, dtype, v) * inv_T - mj);
+    int j = v_off / G + jl;
+    uint32_t x = ebo_draw_word(c->seed, (uint32_t)j >> 2, (uint32_t)l, (uint32_t)s,
+                               bg | ((uint32_t)EBO_STREAM_GROUP << 24), j & 3);
+    double M = mj + log(Sj) + ebo_gumbel(x);
+    if (M > best) { best = M; jbest = jl; }
+  }
+  out->gscore = best;
+  out->sample = -1;
+  if (jbest >= 0) {
+    int lo = jbest * G, hi = lo + G < V_slice ? lo + G : V_slice;
+    double eb = -INFINITY;
+    for (int v = lo; v < hi; ++v) {
+      int vg = v_off + v;
+      uint32_t x = ebo_draw_word(c->seed, (uint32_t)vg >> 2, (uint32_t)l, (uint32_t)s,
+                                 bg | ((uint32_t)EBO_STREAM_GUMBEL << 24), vg & 3);
+      double sc = load_z(row_slice, dtype, v) * inv_T + ebo_gumbel(x);
+      if (sc > eb) { eb = sc; out->sample = vg; }
+    }
+  }
+}
+
+/* The full row's quantities from its slices, given in increasing v_off:
+   the maximum is the largest slice maximum; the sums rescale to it; the
+   argmax is the first slice's argmax that attains it; the draw's winning
+   group is the best slice's (the maximum over groups is the maximum over
+   the slices' maxima; an earlier slice wins an exact tie, as the lower
+   group does), and its element is that slice's. */
+void ebo_combine_slices(const ebo_slice_t* sl, int n, double inv_T, double* H, double* pmax,
+                        int32_t* amax, int32_t* sample) {
+  double M = -INFINITY;
+  int32_t am = -1;
+  for (int i = 0; i < n; ++i)
+    if (sl[i].zmax > M) { M = sl[i].zmax; am = sl[i].amax; }
+  double S = 0.0, W = 0.0;
+  for (int i = 0; i < n; ++i) {
+    if (!(sl[i].zmax > -INFINITY)) continue;
+    double dd = (sl[i].zmax - M) * inv_T;
+    double f = exp(dd);
+    S += f * sl[i].S;
+    W += f * (sl[i].W + dd * sl[i].S);
+  }
+  *H = log(S) - W / S;
+  *pmax = 1.0 / S;
+  *amax = am;
+  double best = -INFINITY;
+  int32_t x = -1;
+  for (int i = 0; i < n; ++i)
+    if (sl[i].gscore > best) { best = sl[i].gscore; x = sl[i].sample; }
+  *sample = x;
+}
+
+/* ------------------------------------------------------------------------- */
 /* Canvas start [NEWS], [DP-INTRO]                                           */
 /* ------------------------------------------------------------------------- */
 

@@ -87,6 +87,19 @@ typedef struct {
                                  differs and pmax >= this; < 0 disables */
 } ebo_config_t;
 
+/* What one vocabulary slice [v_off, v_off + V_slice) of a position's logits
+   contributes when the vocabulary is sharded (one slice per device):
+   its maximum, the sums relative to it, its argmax, and its part of the
+   two-level Gumbel-max draw (best group score and the element drawn in that
+   group), all with global vocabulary indices. */
+typedef struct {
+  double S, W;        /* sum exp(y - y_max), sum exp(y - y_max)(y - y_max) over the slice */
+  double zmax;        /* raw maximum logit of the slice */
+  double gscore;      /* best perturbed group log-partition LSE_j + g_j (-inf if none) */
+  int32_t amax;       /* lowest global id holding zmax */
+  int32_t sample;     /* global id drawn in the best group (-1 if none) */
+} ebo_slice_t;
+
 /* Per-canvas decision margins: how far each decision was from flipping. */
 typedef struct {
   double cum_margin;   /* EB: min |cumulative H - gamma| at the cut (inf if n/a) */
@@ -117,6 +130,10 @@ void ebo_row_stats(const void* row, int dtype, int V, double inv_T,
 /* Two-level Gumbel-max draw for position (b, l) at step s.  Returns the
    sampled vocab id; *margin is the smallest relative top-2 gap of the two
    decisions (group choice, element choice), *group the winning group. */
+void ebo_slice_record(const ebo_config_t* c, const void* row_slice, int dtype, int V_slice,
+                      int v_off, double inv_T, int b, int l, int s, ebo_slice_t* out);
+void ebo_combine_slices(const ebo_slice_t* sl, int n, double inv_T, double* H, double* pmax,
+                        int32_t* amax, int32_t* sample);
 int32_t ebo_sample(const ebo_config_t* c, const void* row, int dtype, double inv_T,
                    int b, int l, int s, double* margin, int32_t* group);
 

@@ -158,6 +158,82 @@ def test_full_parity_neg_inf_logits(E, name, w):
     print(name, stats)
 
 
+def run_split(E, w, bounds, max_resyncs=3):
+    """Vocabulary-sharded logits emulated on one device: one handle per slice
+    (bounds on 64-logit group boundaries), the records stacked in slice order
+    as an all-gather would, slice 0's handle combining; compared with the
+    oracle over the full vocabulary."""
+    handles = []
+    for lo, hi in zip(bounds[:-1], bounds[1:]):
+        cfg = w.sampler_config()
+        handles.append(E.EBSampler(w.B, w.L, hi - lo, device=DEV, vocab_offset=lo,
+                                   vocab_total=w.V, **cfg))
+    h0 = handles[0]
+    canvas, committed, stop = h0.new_canvas()
+    H, amax = h0.outputs()
+    st = O.State(oracle_config(w)).init()
+    torch.cuda.synchronize()
+    assert np.array_equal(canvas.cpu().numpy(), st.canvas)
+    logits = alloc_logits(w)
+    f32 = w.dtype == synth.F32
+    stats = Stats()
+    for s in range(w.num_steps):
+        synth.generate_device(w, s, logits)
+        recs = []
+        for h, (lo, hi) in zip(handles, zip(bounds[:-1], bounds[1:])):
+            r = h.slice_records()
+            h.step_slice(logits[:, :, lo:hi].contiguous(), s, committed, stop, r)
+            recs.append(r)
+        h0.combine(torch.stack(recs), s, canvas, committed, H, amax, stop)
+        smp, pm = h0.draws()
+        torch.cuda.synchronize()
+        lg = host_logits(logits)
+        Hg, amg, cvg, cmg, spg = (H.cpu().numpy(), amax.cpu().numpy(), canvas.cpu().numpy(),
+                                  committed.cpu().numpy(), stop.cpu().numpy())
+        smg, pmg = smp.cpu().numpy(), pm.cpu().numpy()
+        for i in range(w.B):
+            if st.stop[i]:
+                assert spg[i] == st.stop[i] and cmg[i].all()
+                continue
+            out = O.step_canvas(st, i, lg[i], s)
+            compare_rows(stats, i, s, Hg[i], amg[i], pmg[i], smg[i], out, range(w.L), f32,
+                         out["open_before"])
+            differ = bool(np.any((smg[i] != out["sample"]) & out["open_before"]))
+            compare_canvas(stats, st, i, s, (cvg[i], cmg[i], spg[i]), out["margins"], differ)
+        if st.stop.all():
+            break
+    assert st.stop.all()
+    assert stats.resyncs <= max_resyncs, stats
+    for h in handles:
+        assert h.status() == 0
+        h.close()
+    return stats
+
+
+@pytest.mark.parametrize("name,w,bounds", [
+    ("split3_bf16", MID.replace(B=2, num_steps=16, seed=31), [0, 2560, 5120, 8232]),
+    ("split2_f32", MID.replace(B=2, num_steps=12, seed=32, dtype=synth.F32), [0, 4096, 8232]),
+    ("split2_br_greedy", MID.replace(B=2, num_steps=12, seed=33, rule=O.RULE_BR, greedy=1,
+                                     quota=3), [0, 64, 8232]),
+])
+def test_vocabulary_sharded_step_matches_oracle(E, name, w, bounds):
+    stats = run_split(E, w, bounds)
+    print(name, stats)
+
+
+def test_slice_handle_refuses_the_plain_step(E):
+    w = MID.replace(B=1)
+    h = E.EBSampler(w.B, w.L, 4096, device=DEV, vocab_offset=4096, vocab_total=w.V,
+                    **w.sampler_config())
+    canvas, committed, stop = h.new_canvas()
+    H, amax = h.outputs()
+    z = torch.zeros((w.B, w.L, 4096), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(E.EBError):
+        h.step(z, 0, canvas, committed, H, amax, stop)
+    assert int(canvas.max()) < w.V  # the initial canvas covers the whole vocabulary
+    h.close()
+
+
 def test_split_event_times_the_two_kernels(E):
     w = MID.replace(B=1, num_steps=4)
     eb = make_sampler(E, w)

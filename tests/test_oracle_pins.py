@@ -504,3 +504,40 @@ def test_trajectory_invariants(oracle_lib):
                 if st.stop[i]:
                     assert st.committed[i].all()
         assert st.stop.all()  # everything stops by the last step
+
+
+# ----------------------------------------------------------------------------- vocabulary slices
+
+def test_slices_combine_to_the_full_row(oracle_lib):
+    """Vocabulary-sharded logits: the slices' records, combined, give the
+    full row's entropy, max probability, argmax and two-level draw.  Checked
+    against the full-row functions for random partitions on group boundaries,
+    including -inf logits and a slice of -inf only."""
+    rng = np.random.default_rng(31)
+    G = 64
+    for trial in range(60):
+        ng = int(rng.integers(2, 12))
+        V = ng * G - int(rng.integers(0, G))
+        z = rng.normal(0.0, rng.choice([0.5, 3.0]), V)
+        if trial % 3 == 0:
+            z[rng.integers(0, V)] += 15.0
+        if trial % 4 == 1:
+            z[rng.random(V) < 0.2] = -np.inf
+        cuts = sorted(set(rng.choice(np.arange(1, ng), size=int(rng.integers(1, min(4, ng))),
+                                     replace=False).tolist()))
+        bounds = [0] + [c * G for c in cuts] + [V]
+        if trial % 5 == 2:  # one slice of -inf only
+            z[bounds[0]:bounds[1]] = -np.inf
+            z[bounds[-2]] = 1.0  # keep the row finite somewhere
+        cfg = O.Config(B=1, L=4, V=V, group_size=G, seed=int(rng.integers(1 << 30)))
+        inv_T = float(rng.choice([1.0, 1.25, 2.5]))
+        row = z.astype(np.float32)
+        slices = [O.slice_record(cfg, np.ascontiguousarray(row[lo:hi]), lo, inv_T, 0, 2, 7)
+                  for lo, hi in zip(bounds[:-1], bounds[1:])]
+        H, pm, am, x = O.combine_slices(slices, inv_T)
+        H0, pm0, am0, _ = O.row_stats(row, inv_T)
+        x0, margin, _ = O.sample(cfg, row, inv_T, 0, 2, 7)
+        assert am == am0
+        assert abs(H - H0) <= 1e-12 * max(1.0, abs(H0)) and abs(pm - pm0) <= 1e-12
+        if margin > 1e-9:  # not an exact tie between two draws
+            assert x == x0, (trial, x, x0)
