@@ -191,6 +191,12 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint
       : "memory");
 }
 
+// Hint: bring the cache line holding p into L1 (no fault on any address the
+// caller could load).
+__device__ __forceinline__ void prefetch_l1(const void* p) {
+  asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
+}
+
 // Programmatic dependent launch: the dependent grid may be scheduled once
 // every CTA of this grid has signalled (or exited); griddep_wait blocks until
 // the prerequisite grid has completed and its memory operations are visible.

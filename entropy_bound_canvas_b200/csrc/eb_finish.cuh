@@ -199,12 +199,22 @@ __device__ __forceinline__ RowOut finish_row(const StepArgs& a, int bi, int ai, 
     if (NG >= (unsigned long long)a.G1) {
       // every stream CTA owns at least one group, so every CTA from c_first
       // to c_last wrote its records for this row: load four at a time
+      const char* rowp = reinterpret_cast<const char*>(a.logits) + grow * (size_t)a.V * elt_bytes(DT);
       for (int i0 = sl; i0 < nrec; i0 += 4 * TPR) {
         Partial q[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int i = i0 + u * TPR;
           q[u] = i < nrec ? rec[i] : empty_partial();
+        }
+        // every record's top group and draw group may be the row's: start
+        // bringing their logits into L1 while the records merge
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (q[u].agrp != 0x7fffffff)
+            prefetch_l1(rowp + (size_t)q[u].agrp * kGroup * elt_bytes(DT));
+          if (q[u].gidx != 0x7fffffff && !a.greedy)
+            prefetch_l1(rowp + (size_t)q[u].gidx * kGroup * elt_bytes(DT));
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) merge(R, q[u], a.c2);
