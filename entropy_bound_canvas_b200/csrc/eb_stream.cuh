@@ -265,10 +265,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           break;
         }
         if (*(volatile int*)&ctrl->abort) break;
-        if (t.r != row_seen) {
+        const bool new_row = t.r != row_seen;
+        if (new_row) {
           row_seen = t.r;
           bi = act[t.ai];
-          samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
         }
         const char* src = logits + ((size_t)bi * (size_t)a.L + (size_t)t.l) * row_bytes +
                           (size_t)t.j0 * kGroup * elt_bytes(DT);
@@ -280,6 +280,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         const uintptr_t a0 = reinterpret_cast<uintptr_t>(src) & ~(uintptr_t)15;
         const uintptr_t a1 =
             (reinterpret_cast<uintptr_t>(src) + nel * elt_bytes(DT) + 15) & ~(uintptr_t)15;
+        mbar_arrive_expect_tx(&full[st], (uint32_t)(a1 - a0));
+        bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
+                  (uint32_t)(a1 - a0), &full[st], policy);
+        // The position's committed flag is read while the copy is in flight.
+        // Nothing reads the description before the release of `issued`, and
+        // the stage cannot fill before the word producer's arrival, which
+        // follows that release.
+        if (new_row)
+          samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
         TileMeta m;
         m.r = (int)t.r;
         m.j0 = t.j0;
@@ -290,9 +299,6 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         m.delta = (int)(reinterpret_cast<uintptr_t>(src) - a0);
         m.pad = 0;
         meta[st] = m;
-        mbar_arrive_expect_tx(&full[st], (uint32_t)(a1 - a0));
-        bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
-                  (uint32_t)(a1 - a0), &full[st], policy);
         st_release_shared(&ctrl->issued, k + 1);
         ++k;
         if (++st == kStages) {
