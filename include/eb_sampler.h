@@ -135,8 +135,10 @@ typedef struct {
 void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V);
 
 /* Create a sampler on CUDA device `device` (the device must be sm_100).
-   Validates cfg, allocates and zeroes the workspace (partials, tickets,
-   previous argmax, stability counters, per-position draws, status word).
+   Validates cfg, allocates and zeroes the workspace (the per-position
+   partial records of the stream pass, the active-canvas list, previous
+   argmax, stability counters, per-position draws and max probabilities,
+   status word) in one allocation.
    On success *out owns the handle (release with eb_sampler_destroy).
    Errors: INVALID_ARG, OVERFLOW, UNSUPPORTED, OUT_OF_MEMORY, CUDA. */
 int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device);
