@@ -134,6 +134,44 @@ def test_full_parity(E, name, w):
         assert stats.edits > 0, "the editing configuration re-edits some committed token"
 
 
+@pytest.mark.parametrize("name,w", [
+    # one-token vocabulary: every entropy is 0, every canvas commits at step 0
+    ("V1_eb", MID.replace(V=1, L=16, B=2, num_steps=6, seed=41)),
+    ("V1_br_greedy", MID.replace(V=1, L=16, B=2, num_steps=6, seed=45, rule=O.RULE_BR,
+                                 greedy=1, quota=3)),
+    # one position per canvas: the commit rule's minimum of one commits it
+    ("L1", MID.replace(L=1, B=3, V=1000, num_steps=5, seed=42)),
+    # a one-step trajectory: temperature t_max, and the step is the last one
+    ("N1", MID.replace(num_steps=1, B=2, seed=43)),
+    # long canvases: 4 and then 2 finish lanes per position
+    ("L512", MID.replace(L=512, B=1, V=200, num_steps=6, seed=46)),
+    ("L1024_max", MID.replace(L=1024, B=1, V=200, num_steps=6, seed=44)),
+])
+def test_degenerate_shapes(E, name, w):
+    stats = run_full(E, w)
+    print(name, stats)
+
+
+def test_all_canvases_stopped_is_a_no_op(E):
+    w = MID.replace(B=2, seed=47)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    H.fill_(-7.0)
+    amax.fill_(-9)
+    stop.fill_(1)
+    before = (canvas.clone(), committed.clone())
+    logits = alloc_logits(w)
+    for s in range(3):
+        synth.generate_device(w, s, logits)
+        eb.step(logits, s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    assert torch.equal(canvas, before[0]) and torch.equal(committed, before[1])
+    assert (H == -7.0).all() and (amax == -9).all() and (stop == 1).all()
+    assert eb.status() == 0
+    eb.close()
+
+
 def _mask_neg_inf(V):
     """-inf logits, as a vocabulary mask would leave them: a random tenth of the
     vocabulary (new each step), one whole 64-logit group, and the last logit."""
