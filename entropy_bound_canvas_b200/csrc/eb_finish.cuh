@@ -535,7 +535,8 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, FinCtrl* ctrl, const 
   }
 }
 
-// ai: index of canvas bi among the canvases active at the start of the step.
+// act_index[b]: index of canvas b among the canvases active at the start of
+// the step (-1 if it had stopped), written by the stream kernel.
 template <int DT, int TPR>
 __device__ __forceinline__ void finish_rows(const StepArgs& a, const FinLayout& lay,
                                             unsigned char* smem, cgr::cluster_group& cluster,
@@ -564,7 +565,7 @@ __device__ __forceinline__ void finish_rows(const StepArgs& a, const FinLayout& 
 
 template <int DT>
 __global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThreads, 2)
-    finish_kernel(const StepArgs a) {
+    finish_kernel(const StepArgs a, const int32_t* act_index, const int32_t* n_act_ptr) {
   extern __shared__ __align__(128) unsigned char smem[];
   const FinLayout lay = fin_layout(a.L);
   FinCtrl* ctrl = reinterpret_cast<FinCtrl*>(smem + lay.ctrl);
@@ -591,22 +592,12 @@ __global__ void __cluster_dims__(kFinCluster, 1, 1) __launch_bounds__(kFinThread
     }
     if (tid == 0) ctrl->stable_prev = a.stable[bi];
   }
-  // The canvases active in this step are those whose stop flag was clear
-  // when it began, as the stream kernel counted them: this canvas's index
-  // among them and their number, so that no load of what the stream kernel
-  // wrote stands between the wait below and the first record load.
-  int ai = 0, n_act = 0;
-  for (int b0 = 0; b0 < a.B; b0 += kFinThreads) {
-    const int b = b0 + tid;
-    const bool on = b < a.B && __ldcg(a.stop_flags + b) == 0;
-    n_act += __syncthreads_count(on);
-    ai += __syncthreads_count(on && b < bi);
-  }
-  if (__ldcg(a.stop_flags + bi) != 0) ai = -1;
   cluster.sync();  // every CTA of the cluster runs: its shared memory may be written
 
   griddep_wait();  // the stream kernel has completed and its writes are visible
+  const int ai = act_index[bi];
   if (ai < 0) return;  // uniform over the cluster: a stopped canvas is untouched
+  const int n_act = *n_act_ptr;
   const unsigned long long NG =
       (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
   switch (tpr) {

@@ -395,7 +395,9 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   if (h->split_event && cudaEventRecord(h->split_event, st) != cudaSuccess) return EB_ERR_CUDA;
 
   const KernelCfg& kf = h->fin[dtype];
-  void* fargs[] = {&a};
+  const int32_t* act_index = h->act_index;
+  const int32_t* n_act = h->n_act;
+  void* fargs[] = {&a, &act_index, &n_act};
   rc = launch_dependent(kf.fn, dim3(kf.grid), dim3(ebk::kFinThreads), kf.smem, fargs, st);
   if (rc != EB_OK) return rc;
   h->last_step = step;

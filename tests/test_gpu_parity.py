@@ -152,6 +152,16 @@ def test_degenerate_shapes(E, name, w):
     print(name, stats)
 
 
+def test_many_canvases_stopping_at_different_steps(E):
+    """64 canvases: more finish clusters than fit on the GPU at once, so some
+    start after others have run their epilogue and set their stop flags in
+    the same step.  Canvases stop (all committed) between steps 12 and 15."""
+    w = synth.WORKLOADS["serve"].replace(name="many", B=64, L=16, V=1000, seed=48)
+    stats = run_full(E, w)
+    print("many", stats)
+    assert len(set(stats.stop_steps.values())) > 1, "canvases stop at different steps"
+
+
 def test_all_canvases_stopped_is_a_no_op(E):
     w = MID.replace(B=2, seed=47)
     eb = make_sampler(E, w)
