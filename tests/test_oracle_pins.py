@@ -244,6 +244,64 @@ def test_group_draw_uses_group_stream(oracle_lib):
     assert tok == arg and grp == arg
 
 
+def test_argmax_ties_take_the_lowest_index(oracle_lib):
+    """Equal maxima: the argmax is the first of them (within one group, across
+    groups, and across a group boundary)."""
+    V = 300
+    for where in ([5, 6], [5, 200], [63, 64], [0, 299], [130, 131, 140]):
+        row = np.zeros(V, np.float32)
+        row[where] = 3.5
+        _, pmax, amax, _ = O.row_stats(row, 1.0 / 0.8)
+        assert amax == min(where)
+        # k equal maxima of e^(3.5/T) among V - k ones
+        e = math.exp(3.5 / 0.8)
+        assert pmax == pytest.approx(e / (len(where) * e + V - len(where)), rel=1e-12)
+
+
+@pytest.mark.parametrize("k", [1, 3, 64, 100])
+def test_masked_row_is_the_softmax_of_the_finite_logits(oracle_lib, k):
+    """-inf logits drop out: k equal finite logits among -inf ones give
+    H = ln k and pmax = 1/k, the argmax is the first finite one, and no draw
+    lands on a masked token."""
+    V = 500
+    rng = np.random.default_rng(k)
+    finite = np.sort(rng.choice(V, size=k, replace=False))
+    row = np.full(V, -np.inf, np.float32)
+    row[finite] = 1.25
+    for T in (0.4, 1.0):
+        H, pmax, amax, _ = O.row_stats(row, 1.0 / T)
+        assert H == pytest.approx(math.log(k), abs=1e-12)
+        assert pmax == pytest.approx(1.0 / k, rel=1e-12)
+        assert amax == finite[0]
+    cfg = O.Config(B=1, L=4, V=V)
+    drawn = {O.sample(cfg, row, 1.0 / 0.8, 0, l, s)[0] for l in range(4) for s in range(60)}
+    assert drawn <= set(finite.tolist())
+    if k > 1:
+        assert len(drawn) > 1  # equal logits: the draw is not stuck on one token
+
+
+def test_single_token_vocabulary(oracle_lib):
+    """V = 1: entropy 0, pmax 1, argmax 0, and every draw is token 0."""
+    cfg = O.Config(B=1, L=2, V=1)
+    for z in (-3.0, 0.0, 7.5):
+        row = np.array([z], np.float32)
+        H, pmax, amax, _ = O.row_stats(row, 1.0 / 0.4)
+        assert H == 0.0 and pmax == 1.0 and amax == 0
+        assert all(O.sample(cfg, row, 1.0 / 0.4, 0, l, s)[0] == 0 for l in range(2)
+                   for s in range(5))
+
+
+def test_single_finite_logit_is_always_drawn(oracle_lib):
+    V = 1000
+    cfg = O.Config(B=1, L=8, V=V)
+    for j in (0, 63, 64, 999):
+        row = np.full(V, -np.inf, np.float32)
+        row[j] = -40.0
+        assert O.row_stats(row, 1.0)[2] == j
+        assert all(O.sample(cfg, row, 1.0 / 0.8, 0, l, s)[0] == j for l in range(8)
+                   for s in range(4))
+
+
 def test_draw_concentrates_on_dominant_token(oracle_lib):
     z = np.zeros(4096, np.float32)
     z[1234] = 60.0
