@@ -244,6 +244,60 @@ def test_group_draw_uses_group_stream(oracle_lib):
     assert tok == arg and grp == arg
 
 
+def test_element_draw_in_a_later_group_uses_global_ids(oracle_lib):
+    """The element level of the two-level draw, when the winning group is not
+    group 0: recomputed from raw Philox words whose counters carry the GLOBAL
+    vocabulary id v (ctr = (v >> 2, l, s, b), word v & 3).  One group holds
+    logits 40 above every other, so the group level always picks it; a
+    local-id counter (v - 64 j*) would draw other tokens, which the second
+    half of the test checks."""
+    V, G, seed, T = 640, 64, 0x5EED0BADC0FFEE, 0.7
+    rng = np.random.default_rng(17)
+    key = [seed & 0xFFFFFFFF, seed >> 32]
+    n_local_differs = 0
+    for trial in range(24):
+        jstar = 1 + trial % 9  # groups 1 .. 9
+        z = (rng.standard_normal(V) - 40.0).astype(np.float32)
+        z[jstar * G:(jstar + 1) * G] += 40.0
+        l, s, b = trial % 7, 3 + trial, 2 + trial % 5
+        cfg = O.Config(B=8, L=8, V=V, seed=seed, group_size=G)
+        tok, _, grp = O.sample(cfg, z, 1 / T, b, l, s)
+        assert grp == jstar
+
+        def draw(local):
+            best, arg = -np.inf, -1
+            for v in range(jstar * G, (jstar + 1) * G):
+                vc = v - jstar * G if local else v
+                w = int(O.philox4x32_10([vc >> 2, l, s, b], key)[vc & 3])
+                u = (2 * (w >> 9) + 1) * 2.0 ** -24
+                sc = float(z[v]) / T - math.log(-math.log(u))
+                if sc > best:
+                    best, arg = sc, v
+            return arg
+
+        assert tok == draw(local=False)
+        n_local_differs += draw(local=True) != tok
+    assert n_local_differs >= 12  # the pin tells the two counter layouts apart
+
+
+def test_initial_canvas_matches_raw_philox_words(oracle_lib):
+    """Initial canvas token of (b, l): word l & 3 of Philox4x32-10 at
+    ctr = (l >> 2, 0, 0, b | 2 << 24) with b the GLOBAL canvas index
+    (canvas_offset + local index), mapped to (x * V) >> 32; nothing
+    committed, stop flag clear."""
+    for V, seed, off in ((1024, 11, 0), (262144, 0xFEEDFACE12345678, 7), (1000, 3, 1 << 20)):
+        L, B = 37, 3
+        cfg = O.Config(B=B, L=L, V=V, seed=seed, canvas_offset=off)
+        st = O.State(cfg).init()
+        key = [seed & 0xFFFFFFFF, seed >> 32]
+        for bl in range(B):
+            bg = off + bl
+            for l in range(L):
+                w = int(O.philox4x32_10([l >> 2, 0, 0, bg | (2 << 24)], key)[l & 3])
+                assert st.canvas[bl, l] == (w * V) >> 32, (V, bl, l)
+        assert not st.committed.any() and not st.stop.any() and not st.stable.any()
+
+
 def test_argmax_ties_take_the_lowest_index(oracle_lib):
     """Equal maxima: the argmax is the first of them (within one group, across
     groups, and across a group boundary)."""
