@@ -11,13 +11,17 @@ every logit of every active canvas read once, entropies, argmax, draws,
 commit, renoise, stop test.  Each step reads its own 134 MB of logits, more
 than the 126 MB L2, so no step hits in L2 on the previous one's data.
 
-Timing: W eager warm-up steps, then exactly K steps timed with CUDA events on
-the launching stream between a barrier + synchronize on both sides (max over
-ranks); full 48-step trajectories are replayed from one CUDA graph, the
-remainder runs eagerly.  The kernel's own launch durations (for the roofline)
-come from per-launch events over one eager trajectory.  For N > 1 each rank
-runs its own canvas (global canvas index = rank): no data-path collective,
-weak scaling.
+Timing: W eager warm-up steps, then timed regions of exactly K steps, each
+with CUDA events on the launching stream between a barrier + synchronize on
+both sides (max over ranks); the K steps are replayed from CUDA graphs (one
+per full 48-step trajectory, one for the remaining prefix; each starts with
+the canvas init kernel), and the median over the regions is reported.  The
+kernels' own launch durations (for the roofline) come from per-launch events
+over one eager trajectory.  For N > 1 each rank runs its own canvas (global
+canvas index = rank): no data-path collective, weak scaling.
+
+At N = 1 the other large workloads (serve 8x, br 4x, stress 32x fp32) are
+timed afterwards as whole 48-step trajectories and reported under "configs".
 
 --impl reference times the CPU oracle (the float64 restatement in oracle/)
 on the host cores, rank 0 only, on bounded samples of the same workload.
@@ -52,6 +56,11 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--e2e-steps", type=int, default=48)
+    p.add_argument("--repeats", type=int, default=0,
+                   help="timed regions of exactly K steps (median reported); 0 = automatic")
+    p.add_argument("--configs", default="all",
+                   help="other workloads timed after the headline one: all, none, or a list "
+                        "of serve,br,stress (N = 1 only by default)")
     p.add_argument("--profile", action="store_true",
                    help="small case for ncu: logits of steps 0-2 only, three eager steps")
     return p.parse_args()
@@ -206,6 +215,19 @@ def run_reference(args):
 
 # --------------------------------------------------------------------------- our arm
 
+def host_info():
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"host_nproc": os.cpu_count(), "cpu_model": model}
+
+
 def cpu_baseline(w, logits_steps, states):
     """The oracle, as it stands, on full canvas steps at a few step indices."""
     import numpy as np
@@ -223,10 +245,143 @@ def cpu_baseline(w, logits_steps, states):
         t_total += time.perf_counter() - t0
         n_pos += w.L
         used.append(s)
-    return {"value": n_pos / t_total, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{len(used)} full 256-position canvas steps (s = {used[0]}, {used[1]}, ..., "
-                      f"{used[-1]}) of the same trajectory "
-                      f"(single thread, float64), {t_total:.1f} s of CPU work"}
+    out = {"value": n_pos / t_total, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{len(used)} full 256-position canvas steps (s = {used[0]}, {used[1]}, ..., "
+                     f"{used[-1]}) of the same trajectory "
+                     f"(single thread, float64), {t_total:.1f} s of CPU work"}
+    out.update(host_info())
+    return out
+
+
+class Trajectory:
+    """One workload on one device: a sampler handle, its canvas buffers and
+    the logits of every step resident in HBM (or `rotate` buffers reused
+    round-robin when 48 steps of the workload do not fit)."""
+
+    def __init__(self, E, synth, w, dev, rank, rotate=None):
+        import torch
+        self.w, self.dev = w, dev
+        self.N = w.num_steps
+        nbuf = self.N if rotate is None else rotate
+        dt = torch.float32 if w.dtype == synth.F32 else torch.bfloat16
+        self.logits = [torch.empty((w.B, w.L, w.V), dtype=dt, device=dev) for _ in range(nbuf)]
+        for s in range(nbuf):
+            synth.generate_device(w, s, self.logits[s], b0=rank * w.B)
+        self.eb = E.EBSampler(w.B, w.L, w.V, device=dev, canvas_offset=rank * w.B,
+                              **w.sampler_config())
+        self.canvas, self.committed, self.stop = self.eb.new_canvas()
+        self.H, self.amax = self.eb.outputs()
+        self.graphs = {}
+
+    def lg(self, s):
+        return self.logits[s % len(self.logits)]
+
+    def run(self, n):
+        """init + the first n steps, on the current stream."""
+        self.eb.init_canvas(self.canvas, self.committed, self.stop)
+        for s in range(n):
+            self.eb.step(self.lg(s), s, self.canvas, self.committed, self.H, self.amax, self.stop)
+
+    def active_per_step(self):
+        """Active canvases at the start of each step of one trajectory (untimed)."""
+        import torch
+        act = []
+        self.eb.init_canvas(self.canvas, self.committed, self.stop)
+        for s in range(self.N):
+            act.append(int((self.stop == 0).sum().item()))
+            self.eb.step(self.lg(s), s, self.canvas, self.committed, self.H, self.amax, self.stop)
+        torch.cuda.synchronize()
+        return act
+
+    def graph(self, n):
+        """A CUDA graph of init + the first n steps (captured once)."""
+        import torch
+        if n not in self.graphs:
+            g = torch.cuda.CUDAGraph()
+            side = torch.cuda.Stream(self.dev)
+            side.wait_stream(torch.cuda.current_stream(self.dev))
+            with torch.cuda.stream(side):
+                self.run(n)
+                torch.cuda.synchronize()
+                with torch.cuda.graph(g, stream=side):
+                    self.run(n)
+            torch.cuda.synchronize()
+            self.graphs[n] = g
+        return self.graphs[n]
+
+    def kernel_times(self):
+        """Mean per-launch durations (ms) of the step's two kernels over one
+        eager trajectory (steps with an active canvas, step 0 excluded):
+        events before the step, between its kernels (the library's split
+        event) and after it, all on the launching stream."""
+        import torch
+        stream = torch.cuda.current_stream(self.dev)
+        evs = []
+        self.eb.init_canvas(self.canvas, self.committed, self.stop)
+        for s in range(self.N):
+            a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+            self.eb.set_split_event(m)
+            a.record(stream)
+            self.eb.step(self.lg(s), s, self.canvas, self.committed, self.H, self.amax, self.stop)
+            b.record(stream)
+            evs.append((s, a, m, b))
+        self.eb.set_split_event(None)
+        torch.cuda.synchronize()
+        return evs
+
+    def close(self):
+        self.graphs.clear()
+        self.eb.close()
+        self.logits.clear()
+
+
+def timed_regions(replay, repeats, barrier, stream):
+    """Each region: barrier + synchronize, CUDA events around replay(),
+    synchronize + barrier.  Returns the region times in ms."""
+    import torch
+    out = []
+    for _ in range(repeats):
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        replay()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def roofline_of(tr, active, peak, peak_kind):
+    """Stream-kernel roofline of a workload: algorithmic bytes per launch
+    (every logit of the active canvases once) over its event-timed duration."""
+    evs = tr.kernel_times()
+    w = tr.w
+    ks, fs, byts = [], [], []
+    for s, a, m, b in evs:
+        if s == 0 or not active[s]:
+            continue
+        ks.append(a.elapsed_time(m))
+        fs.append(m.elapsed_time(b))
+        byts.append(active[s] * w.L * w.V * w.elt)
+    k_ms = statistics.mean(ks)
+    bytes_launch = statistics.mean(byts)
+    achieved = bytes_launch / (k_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+            "frac": achieved / peak, "kernel": f"ebk::stream_kernel<{'f32' if w.elt == 4 else 'bf16'}>",
+            "kernel_ms": k_ms, "finish_kernel_ms": statistics.mean(fs),
+            "algorithmic_bytes": bytes_launch,
+            "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"}
+
+
+EXTRA = {
+    # name -> (rotate buffers or None, description)
+    "serve": (None, "8 x 256 x 262144 bf16 per GPU, staggered stops, 48 steps resident"),
+    "br": (None, "4 x 256 x 262144 bf16 per GPU, block refinement, greedy, 48 steps resident"),
+    "stress": (3, "32 x 256 x 262144 fp32 per GPU, Zipf-like logits, 3 step buffers "
+                  "rotated (8.6 GB each)"),
+}
 
 
 def run_ours(args):
@@ -254,126 +409,105 @@ def run_ours(args):
         if dist is not None:
             dist.barrier()
 
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+
     w = synth.WORKLOADS[WORKLOAD]
     N = w.num_steps
     K, W = args.steps, max(3, args.warmup)
     stream = torch.cuda.current_stream(dev)
+    peak, peak_kind = peaks()
 
-    # inputs resident in HBM: this rank's canvas for all N steps
-    logits = [torch.empty((w.B, w.L, w.V), dtype=torch.bfloat16, device=dev) for _ in range(N)]
-    for s in range(N):
-        synth.generate_device(w, s, logits[s], b0=rank)
-    eb = E.EBSampler(w.B, w.L, w.V, device=dev, canvas_offset=rank, **w.sampler_config())
-    canvas, committed, stop = eb.new_canvas()
-    H, amax = eb.outputs()
+    tr = Trajectory(E, synth, w, dev, rank)
     torch.cuda.synchronize()
 
     # reference trajectory (untimed): active canvases per step, snapshots for the CPU baseline
     active = []
     snaps = {}
-    eb.init_canvas(canvas, committed, stop)
+    tr.eb.init_canvas(tr.canvas, tr.committed, tr.stop)
     for s in range(N):
-        active.append(int((stop == 0).sum().item()))
+        active.append(int((tr.stop == 0).sum().item()))
         if s % 2 == 0:  # 24 of the 48 steps: about 15 s of oracle work
-            snaps[s] = (canvas[0].cpu().numpy().copy(), committed[0].cpu().numpy().copy(),
-                        amax[0].cpu().numpy().copy())
-        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+            snaps[s] = (tr.canvas[0].cpu().numpy().copy(), tr.committed[0].cpu().numpy().copy(),
+                        tr.amax[0].cpu().numpy().copy())
+        tr.eb.step(tr.lg(s), s, tr.canvas, tr.committed, tr.H, tr.amax, tr.stop)
     torch.cuda.synchronize()
     stop_step = next((s for s in range(N) if s + 1 < N and active[s + 1] == 0), N - 1)
 
     # warm-up: W eager steps along the trajectory
-    eb.init_canvas(canvas, committed, stop)
+    tr.eb.init_canvas(tr.canvas, tr.committed, tr.stop)
     for i in range(W):
         s = i % N
         if s == 0 and i > 0:
-            eb.init_canvas(canvas, committed, stop)
-        eb.step(logits[s], s, canvas, committed, H, amax, stop)
+            tr.eb.init_canvas(tr.canvas, tr.committed, tr.stop)
+        tr.eb.step(tr.lg(s), s, tr.canvas, tr.committed, tr.H, tr.amax, tr.stop)
     torch.cuda.synchronize()
 
-    # one trajectory as a CUDA graph
-    g = torch.cuda.CUDAGraph()
-    side = torch.cuda.Stream(dev)
-    side.wait_stream(stream)
-    with torch.cuda.stream(side):
-        eb.init_canvas(canvas, committed, stop)
-        for s in range(N):
-            eb.step(logits[s], s, canvas, committed, H, amax, stop)
-        torch.cuda.synchronize()
-        with torch.cuda.graph(g, stream=side):
-            eb.init_canvas(canvas, committed, stop)
-            for s in range(N):
-                eb.step(logits[s], s, canvas, committed, H, amax, stop)
-    torch.cuda.synchronize()
-
+    # exactly K steps per timed region: full trajectories and a prefix, each
+    # from a CUDA graph (init + steps), replayed back to back
     full, rem = divmod(K, N)
-    # per step: the stream kernel and the finish kernel; per trajectory: the init kernel
-    launches = full * (2 * N + 1) + (2 * rem + (1 if rem else 0))
-    pos_per_traj = sum(active) * w.L
-    positions = full * pos_per_traj + sum(active[:rem]) * w.L
-    bytes_steps = full * sum(active) + sum(active[:rem])
-    bytes_total = bytes_steps * w.L * w.V * 2
+    g_full = tr.graph(N) if full else None
+    g_rem = tr.graph(rem) if rem else None
+    for _ in range(2):  # warm the graphs
+        if g_full is not None:
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+    torch.cuda.synchronize()
+
+    def region():
+        for _ in range(full):
+            g_full.replay()
+        if g_rem is not None:
+            g_rem.replay()
+
+    launches = full * (2 * N + 1) + ((2 * rem + 1) if rem else 0)
+    positions = full * sum(active) * w.L + sum(active[:rem]) * w.L
+    bytes_total = (full * sum(active) + sum(active[:rem])) * w.L * w.V * w.elt
+    repeats = args.repeats or max(3, min(50, int(0.5 / max(1e-5, K * 40e-6))))
 
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(full):
-        g.replay()
-    if rem:
-        eb.init_canvas(canvas, committed, stop)
-        for s in range(rem):
-            eb.step(logits[s], s, canvas, committed, H, amax, stop)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    barrier()
+    times = timed_regions(region, repeats, barrier, stream)
     clk = clocks.stop()
-    el_ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([el_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        el_ms = float(t.item())
-        p = torch.tensor([positions, bytes_total], device=dev, dtype=torch.float64)
-        dist.all_reduce(p, op=dist.ReduceOp.SUM)
-        positions_all, bytes_all = float(p[0].item()), float(p[1].item())
-    else:
-        positions_all, bytes_all = float(positions), float(bytes_total)
+    el_ms = max_over_ranks(statistics.median(times))
+    positions_all = sum_over_ranks(float(positions))
+    bytes_all = sum_over_ranks(float(bytes_total))
     value = positions_all / (el_ms * 1e-3)
     hbm_gbs_job = bytes_all / (el_ms * 1e-3) / 1e9
 
-    # per-launch durations of the two kernels over one eager trajectory (for
-    # the roofline): events before the step, between its kernels, after it
-    evs = []
-    eb.init_canvas(canvas, committed, stop)
-    for s in range(N):
-        a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-        eb.set_split_event(m)
-        a.record(stream)
-        eb.step(logits[s], s, canvas, committed, H, amax, stop)
-        b.record(stream)
-        evs.append((s, a, m, b))
-    eb.set_split_event(None)
-    torch.cuda.synchronize()
-    durs = [(a.elapsed_time(m), m.elapsed_time(b)) for s, a, m, b in evs if active[s] and s > 0]
-    k_ms = statistics.mean(d for d, _ in durs)
-    fin_ms = statistics.mean(d for _, d in durs)
-    k_bytes = w.B * w.L * w.V * 2  # algorithmic: every logit of the active canvas once
-    achieved = k_bytes / (k_ms * 1e-3) / 1e9
-    peak, peak_kind = peaks()
-    traffic = recorded_traffic()
+    # full-trajectory step time (48 steps) for reference, when the timed region is shorter
+    traj_ms = None
+    if full == 0:
+        g48 = tr.graph(N)
+        traj = timed_regions(g48.replay, 3, barrier, stream)
+        traj_ms = max_over_ranks(statistics.median(traj)) / N
+
+    roof = roofline_of(tr, active, peak, peak_kind)
+    roof["traffic"] = recorded_traffic()
 
     # end-to-end: host (pinned) logits -> device, step, result back to host, every step
     e2e = None
     if not args.no_e2e:
         n_e2e = min(args.e2e_steps, N)
-        host = [logits[s].cpu().pin_memory() for s in range(n_e2e)]
-        dev_buf = torch.empty_like(logits[0])
+        host = [tr.lg(s).cpu().pin_memory() for s in range(n_e2e)]
+        dev_buf = torch.empty_like(tr.lg(0))
         out_cv = torch.empty((w.B, w.L), dtype=torch.int32).pin_memory()
         out_cm = torch.empty((w.B, w.L), dtype=torch.uint8).pin_memory()
         out_sp = torch.empty((w.B,), dtype=torch.uint8).pin_memory()
-        eb.init_canvas(canvas, committed, stop)
+        tr.eb.init_canvas(tr.canvas, tr.committed, tr.stop)
         torch.cuda.synchronize()
         barrier()
         t0 = time.perf_counter()
@@ -382,30 +516,65 @@ def run_ours(args):
         pos_e2e = 0
         for s in range(n_e2e):
             dev_buf.copy_(host[s], non_blocking=True)
-            eb.step(dev_buf, s, canvas, committed, H, amax, stop)
-            out_cv.copy_(canvas, non_blocking=True)
-            out_cm.copy_(committed, non_blocking=True)
-            out_sp.copy_(stop, non_blocking=True)
+            tr.eb.step(dev_buf, s, tr.canvas, tr.committed, tr.H, tr.amax, tr.stop)
+            out_cv.copy_(tr.canvas, non_blocking=True)
+            out_cm.copy_(tr.committed, non_blocking=True)
+            out_sp.copy_(tr.stop, non_blocking=True)
             stream.synchronize()
             pos_e2e += active[s] * w.L
         x1.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = x0.elapsed_time(x1)
-        if dist is not None:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_ms = float(t.item())
-            pos_e2e *= world
+        e2e_ms = max_over_ranks(x0.elapsed_time(x1))
+        pos_e2e = sum_over_ranks(float(pos_e2e))
         e2e = {"value": pos_e2e / (e2e_ms * 1e-3), "unit": UNIT,
-               "h2d_bytes_per_step": w.B * w.L * w.V * 2,
+               "h2d_bytes_per_step": w.B * w.L * w.V * w.elt,
                "d2h_bytes_per_step": w.B * w.L * 4 + w.B * w.L + w.B,
                "steps": n_e2e, "wall_s": time.perf_counter() - t0}
+        del host
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = cpu_baseline(w, logits, snaps)
+        cpu = cpu_baseline(w, tr.logits, snaps)
+    tr.close()
+    del tr
+    torch.cuda.empty_cache()
+
+    # the other large workloads: full 48-step trajectories from one graph each
+    extra = {}
+    names = [] if args.configs == "none" else (
+        list(EXTRA) if args.configs == "all" else args.configs.split(","))
+    if world > 1 and args.configs == "all":
+        names = []  # the scaling runs time the headline workload only
+    for name in names:
+        rotate, desc = EXTRA[name]
+        wx = synth.WORKLOADS[name]
+        tx = Trajectory(E, synth, wx, dev, rank, rotate=rotate)
+        act = tx.active_per_step()
+        gx = tx.graph(wx.num_steps)
+        gx.replay()
+        torch.cuda.synchronize()
+        tx_times = timed_regions(gx.replay, 5, barrier, stream)
+        ms = max_over_ranks(statistics.median(tx_times))
+        pos = sum_over_ranks(float(sum(act) * wx.L))
+        byt = sum_over_ranks(float(sum(act) * wx.L * wx.V * wx.elt))
+        rf = roofline_of(tx, act, peak, peak_kind)
+        gbs = byt / (ms * 1e-3) / 1e9
+        extra[name] = {
+            "workload": desc, "value": pos / (ms * 1e-3), "unit": UNIT,
+            "ms_per_step": ms / wx.num_steps, "steps": wx.num_steps, "repeats": len(tx_times),
+            "active_canvases_per_step": act, "dtype": "f32" if wx.elt == 4 else "bf16",
+            "hbm_gbs": gbs, "hbm_frac_of_peak": gbs / (peak * world),
+            "roofline": {k: rf[k] for k in ("achieved", "frac", "kernel_ms", "finish_kernel_ms",
+                                            "algorithmic_bytes")},
+        }
+        tx.close()
+        del tx, gx
+        torch.cuda.empty_cache()
 
     if rank == 0:
+        timing = (f"each timed region is exactly {K} steps replayed from CUDA graphs "
+                  f"({full} full 48-step trajectories + a {rem}-step prefix, one init kernel "
+                  f"each); {repeats} regions, median reported")
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": el_ms / K, "higher_is_better": True, "scaling": "weak",
@@ -413,26 +582,23 @@ def run_ours(args):
             "config": {
                 "workload": "canvas 1x256x262144 bf16 per GPU, 48-step entropy-bound trajectory",
                 "B_per_gpu": w.B, "L": w.L, "V": w.V, "num_steps": N, "seed": w.seed,
-                "stop_step": stop_step,
+                "stop_step": stop_step, "repeats": repeats,
                 "l2": "inputs larger than L2: each step reads its own 134 MB of logits",
-                "timing": "full 48-step trajectories replayed from one CUDA graph, remainder eager",
+                "timing": timing,
             },
             "hbm_gbs": hbm_gbs_job,
             "hbm_frac_of_peak": hbm_gbs_job / (peak * world),
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": traffic,
-                         "kernel": "ebk::stream_kernel<bf16>",
-                         "kernel_ms": k_ms, "finish_kernel_ms": fin_ms,
-                         "algorithmic_bytes": k_bytes,
-                         "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"},
+            "trajectory_ms_per_step": traj_ms,
+            "region_ms": {"median": statistics.median(times), "min": min(times),
+                          "max": max(times)},
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
             "clocks": clk,
+            "configs": extra,
         }
         print(json.dumps(line), flush=True)
-    del g
-    eb.close()
     if dist is not None:
         dist.destroy_process_group()
 
