@@ -61,6 +61,9 @@ def parse():
     p.add_argument("--configs", default="all",
                    help="other workloads timed after the headline one: all, none, or a list "
                         "of serve,br,stress (N = 1 only by default)")
+    p.add_argument("--split-v", action="store_true",
+                   help="vocabulary-sharded canvas: each rank holds a slice of the vocabulary; "
+                        "a step is the slice pass, one all-gather of the records, the combine")
     p.add_argument("--profile", action="store_true",
                    help="small case for ncu: logits of steps 0-2 only, three eager steps")
     return p.parse_args()
@@ -603,6 +606,95 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+def run_split_v(args):
+    """The canvas workload with its vocabulary split over the ranks (a
+    tensor-parallel LM head): rank r holds a contiguous, group-aligned slice
+    of every row; each step runs the slice pass on every rank, one NCCL
+    all-gather of the per-position records and the combine.  Total work is
+    fixed, so this is strong scaling.  Eager steps (the collective is not
+    captured), timed with CUDA events between barriers, max over ranks."""
+    import torch
+
+    import entropy_bound_canvas_b200 as E
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    w = synth.WORKLOADS[WORKLOAD]
+    N = w.num_steps
+    K, W = args.steps, max(3, args.warmup)
+    ng = (w.V + 63) // 64
+    per = (ng + world - 1) // world
+    lo, hi = min(ng, rank * per) * 64, min(w.V, min(ng, (rank + 1) * per) * 64)
+    full = torch.empty((w.B, w.L, w.V), dtype=torch.bfloat16, device=dev)
+    sl = []
+    for s in range(N):
+        synth.generate_device(w, s, full)
+        sl.append(full[:, :, lo:hi].contiguous())
+    del full
+    torch.cuda.empty_cache()
+    eb = E.EBSampler(w.B, w.L, hi - lo, device=dev, vocab_offset=lo, vocab_total=w.V,
+                     **w.sampler_config())
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    group = None
+
+    def run(n):
+        eb.init_canvas(canvas, committed, stop)
+        for s in range(n):
+            eb.step_split(sl[s % N], s % N, canvas, committed, H, amax, stop, group=group)
+
+    run(W)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream(dev)
+    full_t, rem = divmod(K, N)
+
+    def region():
+        for _ in range(full_t):
+            run(N)
+        if rem:
+            run(rem)
+
+    times = timed_regions(region, 3, barrier, stream)
+    el = statistics.median(times)
+    if dist is not None:
+        t = torch.tensor([el], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        el = float(t.item())
+    positions = K * w.L * w.B
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": positions / (el * 1e-3), "unit": UNIT, "n_gpus": world,
+            "steps": K, "warmup": W, "ms_per_step": el / K, "higher_is_better": True,
+            "scaling": "strong", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "canvas 1x256x262144 bf16, vocabulary split over the ranks",
+                       "slice_width": hi - lo, "collective": "all_gather_into_tensor (NCCL)",
+                       "timing": "eager steps (slice pass, all-gather, combine), median of 3 "
+                                 "regions of exactly K steps"},
+            "gpu_launches": K * 2 + (full_t + (1 if rem else 0)),
+        }
+        print(json.dumps(line), flush=True)
+    eb.close()
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_profile_case():
     """Three eager steps of the benchmark workload (about 0.4 GB on the device)."""
     import torch
@@ -632,6 +724,8 @@ def main():
         return
     if args.impl == "reference":
         run_reference(args)
+    elif args.split_v:
+        run_split_v(args)
     else:
         run_ours(args)
 

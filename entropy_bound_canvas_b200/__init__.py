@@ -92,6 +92,8 @@ def _lib():
         L.eb_slice_record_bytes.restype = C.c_size_t
         L.eb_sampler_set_split_event.argtypes = [vp, vp]
         L.eb_sampler_set_split_event.restype = i32
+        L.eb_sampler_set_wait_limit.argtypes = [vp, C.c_uint64]
+        L.eb_sampler_set_wait_limit.restype = i32
         L.eb_sampler_workspace_bytes.argtypes = [vp]
         L.eb_sampler_workspace_bytes.restype = C.c_size_t
         L.eb_sampler_destroy.argtypes = [vp]
@@ -339,6 +341,13 @@ class EBSampler:
                 event.record(_torch().cuda.current_stream(self.device))
             ptr = C.c_void_p(event.cuda_event)
         _check(_lib().eb_sampler_set_split_event(self._h, ptr), "eb_sampler_set_split_event")
+
+    def set_wait_limit(self, limit_ns: int = 0):
+        """Limit (ns) of the stream kernel's pipeline waits; 0 = the default
+        2 s.  A diagnostic hook: a tiny limit makes a wait run out, which sets
+        STATUS_TIMEOUT instead of hanging (see include/eb_sampler.h)."""
+        _check(_lib().eb_sampler_set_wait_limit(self._h, int(limit_ns)),
+               "eb_sampler_set_wait_limit")
 
     def workspace_bytes(self) -> int:
         return int(_lib().eb_sampler_workspace_bytes(self._h))

@@ -136,17 +136,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Every wait on a barrier gives up after this long and reports a timeout.
+// Every wait gives up after a limit and reports a timeout: the pipeline
+// waits after the step's configured limit (2 s unless a test shortens it),
+// the drain of copies still in flight at a kernel's exit after kDrainLimitNs.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
+constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -161,7 +165,8 @@ __device__ __forceinline__ int ld_acquire_shared(const int* p) {
 }
 
 // Waits (bounded like mbar_wait) until *p > k.
-__device__ __forceinline__ bool wait_counter_above(const int* p, int k) {
+__device__ __forceinline__ bool wait_counter_above(const int* p, int k,
+                                                   uint64_t limit_ns = kWaitLimitNs) {
   if (ld_acquire_shared(p) > k) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
@@ -170,8 +175,30 @@ __device__ __forceinline__ bool wait_counter_above(const int* p, int k) {
       __nanosleep(32);
       if (ld_acquire_shared(p) > k) return true;
     }
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Waits (bounded) until *p == v.
+__device__ __forceinline__ bool wait_counter_equal(const int* p, int v,
+                                                   uint64_t limit_ns = kWaitLimitNs) {
+  if (ld_acquire_shared(p) == v) return true;
+  const uint64_t t0 = global_ns();
+  for (;;) {
+#pragma unroll 1
+    for (int i = 0; i < 32; ++i) {
+      __nanosleep(20);
+      if (ld_acquire_shared(p) == v) return true;
+    }
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// Shared-memory add with release semantics (publishes this thread's earlier
+// shared-memory writes to a thread that reads the counter with acquire).
+__device__ __forceinline__ void red_release_shared_add(int* p, int v) {
+  asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
+               : "memory");
 }
 
 // L2 policy for data read exactly once: evict it first, so that a stream

@@ -2,10 +2,11 @@
 //
 // Validation, the device workspace, launch configuration and error codes.
 // A step is two kernels on the caller's stream: the persistent stream kernel
-// (eb_stream.cuh, one CTA per SM) and the finish kernel
-// (eb_finish.cuh, one 8-CTA cluster per canvas), launched as a programmatic
-// dependent of the first so that its launch overlaps the first one's end.
-// All the per-step arithmetic runs in those kernels.
+// (eb_stream.cuh, one CTA per SM: every logit once, and every position's
+// entropy, argmax, max probability and draw) and the epilogue kernel
+// (eb_finish.cuh, one CTA per canvas: the canvas decisions), launched as a
+// programmatic dependent of the first so that its launch overlaps the first
+// one's end.  All the per-step arithmetic runs in those kernels.
 #include "eb_sampler.h"
 
 #include <cuda_runtime.h>
@@ -23,7 +24,7 @@
 
 namespace {
 
-using ebk::Partial;
+using ebk::Rec;
 using ebk::StepArgs;
 
 struct KernelCfg {
@@ -31,6 +32,60 @@ struct KernelCfg {
   size_t smem = 0;
   int grid = 0;
 };
+
+constexpr int kMaxDevices = 64;
+
+// Kernel attributes are process-wide per device: the stream kernels'
+// dynamic shared memory opt-in is set once per device to the device maximum,
+// so that no handle ever lowers a value another handle relies on.
+struct DeviceAttrs {
+  std::once_flag once;
+  int rc = EB_ERR_CUDA;
+  int sms = 0;
+  size_t optin = 0;
+};
+DeviceAttrs g_dev[kMaxDevices];
+
+void device_setup(DeviceAttrs& d, int device) {
+  int sms = 0, optin = 0, major = 0;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
+      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
+          cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess) {
+    cudaGetLastError();
+    d.rc = EB_ERR_CUDA;
+    return;
+  }
+  if (major != 10) {
+    d.rc = EB_ERR_UNSUPPORTED;
+    return;
+  }
+  if (cudaFuncSetAttribute(ebk::stream_kernel<ebk::kF32>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::stream_kernel<ebk::kBF16>,
+                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess) {
+    cudaGetLastError();
+    d.rc = EB_ERR_CUDA;
+    return;
+  }
+  d.sms = sms;
+  d.optin = (size_t)optin;
+  d.rc = EB_OK;
+}
+
+// The current device's attributes, set up on first use (the device must be
+// current).
+int device_attrs(int device, DeviceAttrs** out) {
+  if (device < 0 || device >= kMaxDevices) return EB_ERR_UNSUPPORTED;
+  DeviceAttrs& d = g_dev[device];
+  std::call_once(d.once, device_setup, std::ref(d), device);
+  *out = &d;
+  return d.rc;
+}
 
 }  // namespace
 
@@ -40,16 +95,17 @@ struct eb_sampler {
   int sms = 0;
   int ng = 0;
   int max_segs = 0;  // stream CTAs that can share one row
-  int nw = 0;        // records per (row, stream CTA)
-  KernelCfg k[2];     // stream kernel [dtype]
-  KernelCfg fin[2];   // finish kernel [dtype]
+  KernelCfg k[2];    // stream kernel [dtype]
+  KernelCfg epi;     // epilogue kernel
   KernelCfg combine;  // combine kernel (vocabulary slices)
   int V_tot = 0;      // global vocabulary size
   int slice_step = -1;
+  uint64_t wait_ns = ebk::kWaitLimitNs;
   // workspace (one allocation)
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  Partial* partials = nullptr;
+  Rec* recs = nullptr;
+  int32_t* row_cnt = nullptr;
   uint32_t* status = nullptr;
   int32_t* act_index = nullptr;
   int32_t* n_act = nullptr;
@@ -106,52 +162,36 @@ int validate_config(const eb_config_t* c) {
   return EB_OK;
 }
 
+// One persistent CTA per SM, fewer if there are fewer stage-sized tiles.
 template <int DT>
-int setup_kernel(eb_sampler* h, const cudaDeviceProp& prop) {
+int stream_grid(int sms, uint64_t groups) {
+  const uint64_t want = (groups + ebk::StreamShape<DT>::kStageGroups - 1) /
+                        ebk::StreamShape<DT>::kStageGroups;
+  return (int)std::min<uint64_t>((uint64_t)sms, std::max<uint64_t>(1, want));
+}
+
+// Most stream CTAs one row can span when each owns at least
+// floor(rows ng / G) groups: floor((ng - 1) G / (rows ng)) + 2, at most G.
+int row_max_segs(int G, uint64_t rows, int ng) {
+  const uint64_t Lng = rows * (uint64_t)ng;
+  const uint64_t segs = ((uint64_t)(ng - 1) * (uint64_t)G) / Lng + 2;
+  return (int)std::min<uint64_t>((uint64_t)G, segs);
+}
+
+template <int DT>
+int setup_kernel(eb_sampler* h, const DeviceAttrs& d) {
   KernelCfg& kc = h->k[DT];
-  const ebk::StreamLayout lay = ebk::stream_layout<DT>(h->cfg.B);
   kc.fn = reinterpret_cast<const void*>(&ebk::stream_kernel<DT>);
-  kc.smem = lay.total;
-  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
-  if (cudaFuncSetAttribute(ebk::stream_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kc.smem) != cudaSuccess)
-    return EB_ERR_CUDA;
+  kc.smem = ebk::stream_layout<DT>(h->cfg.B).total;
+  if (kc.smem > d.optin) return EB_ERR_OVERFLOW;
   int per_sm = 0;
   if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ebk::stream_kernel<DT>,
                                                     ebk::StreamShape<DT>::kThreads, kc.smem) !=
           cudaSuccess ||
       per_sm < 1)
     return EB_ERR_CUDA;
-  // one persistent CTA per SM, fewer if there are fewer stage-sized tiles
   const uint64_t groups = (uint64_t)h->cfg.B * (uint64_t)h->cfg.L * (uint64_t)h->ng;
-  const uint64_t want = (groups + ebk::StreamShape<DT>::kStageGroups - 1) /
-                        ebk::StreamShape<DT>::kStageGroups;
-  kc.grid = (int)std::min<uint64_t>((uint64_t)prop.multiProcessorCount, std::max<uint64_t>(1, want));
-  return EB_OK;
-}
-
-template <int DT>
-int setup_finish(eb_sampler* h, const cudaDeviceProp& prop) {
-  KernelCfg& kc = h->fin[DT];
-  kc.fn = reinterpret_cast<const void*>(&ebk::finish_kernel<DT>);
-  kc.smem = ebk::fin_layout(h->cfg.L).total;
-  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
-  if (cudaFuncSetAttribute(ebk::finish_kernel<DT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kc.smem) != cudaSuccess)
-    return EB_ERR_CUDA;
-  kc.grid = h->cfg.B * ebk::kFinCluster;
-  return EB_OK;
-}
-
-int setup_combine(eb_sampler* h, const cudaDeviceProp& prop) {
-  KernelCfg& kc = h->combine;
-  kc.fn = reinterpret_cast<const void*>(&ebk::combine_kernel<ebk::kBF16>);
-  kc.smem = ebk::fin_layout(h->cfg.L).total;
-  if (kc.smem > (size_t)prop.sharedMemPerBlockOptin) return EB_ERR_OVERFLOW;
-  if (cudaFuncSetAttribute(ebk::combine_kernel<ebk::kBF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kc.smem) != cudaSuccess)
-    return EB_ERR_CUDA;
-  kc.grid = h->cfg.B * ebk::kFinCluster;
+  kc.grid = stream_grid<DT>(d.sms, groups);
   return EB_OK;
 }
 
@@ -192,39 +232,42 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   if (device < 0 || device >= ndev) return EB_ERR_INVALID_ARG;
   DeviceGuard guard(device);
   if (!guard.ok) return EB_ERR_CUDA;
-  cudaDeviceProp prop;
-  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess) return EB_ERR_CUDA;
-  if (prop.major != 10) return EB_ERR_UNSUPPORTED;
+  DeviceAttrs* d = nullptr;
+  if ((rc = device_attrs(device, &d)) != EB_OK) return rc;
 
   eb_sampler* h = new (std::nothrow) eb_sampler();
   if (!h) return EB_ERR_OUT_OF_MEMORY;
   h->cfg = *cfg;
   h->device = device;
-  h->sms = prop.multiProcessorCount;
+  h->sms = d->sms;
   h->ng = (int)(((int64_t)cfg->V + ebk::kGroup - 1) / ebk::kGroup);
 
-  if ((rc = setup_kernel<ebk::kF32>(h, prop)) != EB_OK ||
-      (rc = setup_kernel<ebk::kBF16>(h, prop)) != EB_OK ||
-      (rc = setup_finish<ebk::kF32>(h, prop)) != EB_OK ||
-      (rc = setup_finish<ebk::kBF16>(h, prop)) != EB_OK || (rc = setup_combine(h, prop)) != EB_OK) {
+  if ((rc = setup_kernel<ebk::kF32>(h, *d)) != EB_OK ||
+      (rc = setup_kernel<ebk::kBF16>(h, *d)) != EB_OK) {
     delete h;
     return rc;
   }
+  h->epi.fn = reinterpret_cast<const void*>(&ebk::epilogue_kernel);
+  h->epi.smem = ebk::epi_layout(cfg->L).total;
+  h->epi.grid = cfg->B;
+  h->combine.fn = reinterpret_cast<const void*>(&ebk::combine_kernel);
+  h->combine.smem = h->epi.smem;
+  h->combine.grid = cfg->B;
+  if (h->epi.smem > d->optin) {
+    delete h;
+    return EB_ERR_OVERFLOW;
+  }
   h->V_tot = cfg->vocab_total > 0 ? cfg->vocab_total : cfg->V;
-  // Most CTAs one row can span: with one active canvas each CTA owns at
-  // least floor(L ng / G) groups, so a row meets at most
-  // floor((ng - 1) G / (L ng)) + 2 of them.
   int gmax = 0;
-  for (int d = 0; d < 2; ++d) gmax = std::max(gmax, h->k[d].grid);
-  const uint64_t Lng = (uint64_t)cfg->L * (uint64_t)h->ng;
-  const uint64_t segs = ((uint64_t)(h->ng - 1) * (uint64_t)gmax) / Lng + 2;
-  h->max_segs = (int)std::min<uint64_t>((uint64_t)gmax, segs);
-  h->nw = ebk::stream_consumer_warps();
+  for (int k = 0; k < 2; ++k) gmax = std::max(gmax, h->k[k].grid);
+  h->max_segs = row_max_segs(gmax, (uint64_t)cfg->L, h->ng);
 
   const size_t BL = (size_t)cfg->B * (size_t)cfg->L;
   size_t off = 0;
-  const size_t o_part = off;
-  off = align256(off + sizeof(Partial) * BL * (size_t)h->max_segs * (size_t)h->nw);
+  const size_t o_rec = off;
+  off = align256(off + sizeof(Rec) * BL * (size_t)h->max_segs);
+  const size_t o_cnt = off;
+  off = align256(off + sizeof(int32_t) * BL);
   const size_t o_status = off;
   off = align256(off + sizeof(uint32_t));
   const size_t o_act = off;
@@ -249,7 +292,8 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
     return EB_ERR_CUDA;
   }
   char* base = static_cast<char*>(h->ws);
-  h->partials = reinterpret_cast<Partial*>(base + o_part);
+  h->recs = reinterpret_cast<Rec*>(base + o_rec);
+  h->row_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
   h->status = reinterpret_cast<uint32_t*>(base + o_status);
   h->act_index = reinterpret_cast<int32_t*>(base + o_act);
   h->n_act = h->act_index + cfg->B;
@@ -268,7 +312,7 @@ int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
   if (!guard.ok) return EB_ERR_CUDA;
   const eb_config_t& c = h->cfg;
   ebk::init_canvas_kernel<<<c.B, 256, 0, (cudaStream_t)stream>>>(
-      canvas, committed, stop_flags, h->stable, c.L, h->V_tot, c.canvas_offset,
+      canvas, committed, stop_flags, h->stable, h->row_cnt, c.L, h->V_tot, c.canvas_offset,
       (uint32_t)(c.seed & 0xffffffffu), (uint32_t)(c.seed >> 32));
   if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = -1;
@@ -294,7 +338,8 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
   const eb_config_t& c = h->cfg;
   const double T = step_temperature(c, step);
   std::memset(&a, 0, sizeof(a));
-  a.partials = h->partials;
+  a.recs = h->recs;
+  a.row_cnt = h->row_cnt;
   a.prev_amax = h->prev_amax;
   a.stable = h->stable;
   a.sample = h->sample;
@@ -302,6 +347,7 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
   a.status = h->status;
   a.act_index = h->act_index;
   a.n_act = h->n_act;
+  a.wait_ns = h->wait_ns;
   a.B = c.B;
   a.L = c.L;
   a.V = c.V;
@@ -309,7 +355,6 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
   a.s = step;
   a.N = c.num_steps;
   a.max_segs = h->max_segs;
-  a.nw = h->nw;
   a.rule = c.rule;
   a.quota = c.quota;
   a.stability_steps = c.stability_steps;
@@ -329,11 +374,11 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
 }
 
 // The stream kernel over `logits` (this device's rows or vocabulary slice).
-int launch_stream(eb_sampler* h, StepArgs& a, const void* logits, int dtype, cudaStream_t st) {
+int launch_stream(const KernelCfg& kc, StepArgs& a, const void* logits, int dtype, size_t V,
+                  cudaStream_t st) {
   const size_t elt = dtype == EB_F32 ? 4 : 2;
   a.logits = logits;
-  a.vec_ok = ((uintptr_t)logits % 16 == 0) && (((size_t)h->cfg.V * elt) % 16 == 0) ? 1 : 0;
-  const KernelCfg& kc = h->k[dtype];
+  a.vec_ok = ((uintptr_t)logits % 16 == 0) && ((V * elt) % 16 == 0) ? 1 : 0;
   a.G1 = kc.grid;
   void* args[] = {&a};
   if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), args, kc.smem, st) !=
@@ -389,16 +434,15 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.H_out = entropies;
   a.amax_out = argmax;
   a.stop_flags = stop_flags;
-  int rc = launch_stream(h, a, logits, dtype, st);
+  int rc = launch_stream(h->k[dtype], a, logits, dtype, (size_t)c.V, st);
   if (rc != EB_OK) return rc;
 
   if (h->split_event && cudaEventRecord(h->split_event, st) != cudaSuccess) return EB_ERR_CUDA;
 
-  const KernelCfg& kf = h->fin[dtype];
   const int32_t* act_index = h->act_index;
-  const int32_t* n_act = h->n_act;
-  void* fargs[] = {&a, &act_index, &n_act};
-  rc = launch_dependent(kf.fn, dim3(kf.grid), dim3(ebk::kFinThreads), kf.smem, fargs, st);
+  void* eargs[] = {&a, &act_index};
+  rc = launch_dependent(h->epi.fn, dim3(h->epi.grid), dim3(ebk::kEpiThreads), h->epi.smem, eargs,
+                        st);
   if (rc != EB_OK) return rc;
   h->last_step = step;
   return EB_OK;
@@ -422,16 +466,8 @@ int eb_sampler_step_slice(eb_sampler_t* h, const void* logits, int dtype, int st
   fill_args(h, a, step);
   a.committed = const_cast<uint8_t*>(committed);  // read only on this path
   a.stop_flags = const_cast<uint8_t*>(stop_flags);
-  int rc = launch_stream(h, a, logits, dtype, st);
-  if (rc != EB_OK) return rc;
-  const int32_t* act_index = h->act_index;
-  const int32_t* n_act = h->n_act;
-  ebk::SliceRecord* rec = static_cast<ebk::SliceRecord*>(records);
-  void* sargs[] = {&a, &act_index, &n_act, &rec};
-  const void* fn = dtype == EB_F32 ? reinterpret_cast<const void*>(&ebk::slice_finish_kernel<ebk::kF32>)
-                                   : reinterpret_cast<const void*>(&ebk::slice_finish_kernel<ebk::kBF16>);
-  rc = launch_dependent(fn, dim3((unsigned)((c.L + 31) / 32), (unsigned)c.B), dim3(256), 0, sargs,
-                        st);
+  a.slice_out = static_cast<ebk::SliceRecord*>(records);
+  const int rc = launch_stream(h->k[dtype], a, logits, dtype, (size_t)c.V, st);
   if (rc != EB_OK) return rc;
   h->slice_step = step;
   return EB_OK;
@@ -461,7 +497,7 @@ int eb_sampler_combine(eb_sampler_t* h, const void* records, int n_slices, int s
   const int32_t* act_index = h->act_index;
   const ebk::SliceRecord* rec = static_cast<const ebk::SliceRecord*>(records);
   void* cargs[] = {&a, &act_index, &rec, &n_slices};
-  if (cudaLaunchKernel(h->combine.fn, dim3(h->combine.grid), dim3(ebk::kFinThreads), cargs,
+  if (cudaLaunchKernel(h->combine.fn, dim3(h->combine.grid), dim3(ebk::kEpiThreads), cargs,
                        h->combine.smem, st) != cudaSuccess)
     return EB_ERR_CUDA;
   h->last_step = step;
@@ -561,6 +597,12 @@ int eb_sampler_set_split_event(eb_sampler_t* h, void* event) {
   return EB_OK;
 }
 
+int eb_sampler_set_wait_limit(eb_sampler_t* h, uint64_t limit_ns) {
+  if (!h) return EB_ERR_INVALID_ARG;
+  h->wait_ns = limit_ns == 0 ? ebk::kWaitLimitNs : limit_ns;
+  return EB_OK;
+}
+
 size_t eb_sampler_workspace_bytes(const eb_sampler_t* h) { return h ? h->ws_bytes : 0; }
 
 void eb_sampler_destroy(eb_sampler_t* h) {
@@ -586,7 +628,7 @@ const char* eb_strerror(int code) {
   }
 }
 
-int eb_version(void) { return 102; }
+int eb_version(void) { return 200; }
 
 }  // extern "C"
 
@@ -595,38 +637,31 @@ int eb_version(void) { return 102; }
 //
 // For callers that cannot or must not allocate device memory (a hard memory
 // budget, a plugin given raw pointers, no sampler handle): the stream pass's
-// partial records live in a static device array instead of a workspace.
+// records, row counters and per-row side outputs live in a static device
+// array instead of a workspace.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr size_t kNoAllocCtrlBytes = 256;  // stop flag, status, active index, count
-constexpr int kNoAllocMaxDevices = 64;
 
 }  // namespace
 
-// Scratch: [0, 256) control words (must start at zero: the stop flag of the
-// single pseudo-canvas and the status word; the active index and count are
-// written by the stream kernel), then the partial records.
+// Scratch: [0, 256) control words (the stop flag of the single pseudo-canvas
+// and the status word must start at zero; the active index and count are
+// written by the stream kernel), then the row records, the row counters
+// (zero at the start of every call) and the per-row max probability and
+// draw the stream kernel also writes.
 static __device__ __align__(256) unsigned char g_noalloc_scratch[EB_NOALLOC_SCRATCH_BYTES];
 
 namespace ebk {
 
-// One 8-lane subgroup per row: the finish kernel's per-position reduction
-// (record merge, exact top group), without the draw and the canvas epilogue.
-template <int DT>
-__global__ void __launch_bounds__(256) row_stats_kernel(const StepArgs a,
-                                                        const int32_t* n_act_ptr) {
-  constexpr int kTPR = 8;
-  const int tid = threadIdx.x;
-  const int row = blockIdx.x * (256 / kTPR) + tid / kTPR;
-  const int sl = tid % kTPR;
-  const bool valid = row < a.L;
-  const unsigned long long NG =
-      (unsigned long long)(*n_act_ptr) * (unsigned long long)a.L * (unsigned long long)a.ng;
-  const RowOut ro = finish_row<DT, kTPR>(a, 0, 0, valid ? row : 0, valid, false, sl, NG);
-  if (valid && sl == 0) {
-    a.H_out[row] = ro.H;
-    a.amax_out[row] = ro.amax;
+// After the stream pass: if a wait of that pass gave up (status word set),
+// every row's outputs are marked invalid rather than left stale.
+__global__ void noalloc_mark_kernel(const uint32_t* status, float* H, int32_t* amax, int rows) {
+  if (__ldcg(status) == 0u) return;
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < rows; i += gridDim.x * blockDim.x) {
+    H[i] = __int_as_float(0x7fc00000);
+    amax[i] = -1;
   }
 }
 
@@ -638,77 +673,56 @@ struct NoAllocDevice {
   std::once_flag once;
   int rc = EB_ERR_CUDA;
   unsigned char* scratch = nullptr;
-  int sms = 0;
 };
-NoAllocDevice g_noalloc_dev[kNoAllocMaxDevices];
+NoAllocDevice g_noalloc_dev[kMaxDevices];
 
-// Once per device: the scratch's device address and the stream kernel's
-// shared-memory opt-in (set to the device maximum, so that it never lowers
-// a value a sampler handle set for a larger active list).
-void noalloc_setup(NoAllocDevice& d, int device) {
+// Once per device (the device current): the scratch's device address.
+void noalloc_setup(NoAllocDevice& d) {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) {
     cudaGetLastError();
     d.rc = EB_ERR_CUDA;
     return;
   }
-  int sms = 0, optin = 0, major = 0;
-  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, device) != cudaSuccess ||
-      cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, device) !=
-          cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, device) != cudaSuccess) {
-    d.rc = EB_ERR_CUDA;
-    return;
-  }
-  if (major != 10) {
-    d.rc = EB_ERR_UNSUPPORTED;
-    return;
-  }
-  if ((size_t)optin < ebk::stream_layout<ebk::kF32>(1).total ||
-      (size_t)optin < ebk::stream_layout<ebk::kBF16>(1).total) {
-    d.rc = EB_ERR_OVERFLOW;
-    return;
-  }
-  if (cudaFuncSetAttribute(ebk::stream_kernel<ebk::kF32>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
-      cudaFuncSetAttribute(ebk::stream_kernel<ebk::kBF16>,
-                           cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess) {
-    d.rc = EB_ERR_CUDA;
-    return;
-  }
   d.scratch = static_cast<unsigned char*>(p);
-  d.sms = sms;
   d.rc = EB_OK;
 }
 
 template <int DT>
-int noalloc_launch(const NoAllocDevice& d, const void* logits, int32_t rows, int32_t V,
-                   double T, float* entropies, int32_t* argmax, cudaStream_t st) {
+int noalloc_launch(const NoAllocDevice& nd, const DeviceAttrs& d, const void* logits, int32_t rows,
+                   int32_t V, double T, float* entropies, int32_t* argmax, cudaStream_t st) {
   using Sh = ebk::StreamShape<DT>;
   const int ng = (int)(((int64_t)V + ebk::kGroup - 1) / ebk::kGroup);
   const uint64_t groups = (uint64_t)rows * (uint64_t)ng;
-  const uint64_t want = (groups + Sh::kStageGroups - 1) / Sh::kStageGroups;
-  const int grid = (int)std::min<uint64_t>((uint64_t)d.sms, std::max<uint64_t>(1, want));
-  // stream CTAs a row can meet (each CTA owns at least floor(groups / grid))
-  const uint64_t segs = ((uint64_t)(ng - 1) * (uint64_t)grid) / groups + 2;
-  const int max_segs = (int)std::min<uint64_t>((uint64_t)grid, segs);
-  const int nw = ebk::stream_consumer_warps();
-  const uint64_t rec_bytes =
-      (uint64_t)rows * (uint64_t)max_segs * (uint64_t)nw * (uint64_t)sizeof(Partial);
-  if (rec_bytes > EB_NOALLOC_SCRATCH_BYTES - kNoAllocCtrlBytes) return EB_ERR_OVERFLOW;
+  const int grid = stream_grid<DT>(d.sms, groups);
+  const int max_segs = row_max_segs(grid, (uint64_t)rows, ng);
+  const uint64_t rec_bytes = (uint64_t)rows * (uint64_t)max_segs * (uint64_t)sizeof(Rec);
+  const uint64_t side_bytes = (uint64_t)rows * 12u;  // counter, pmax, draw
+  if (kNoAllocCtrlBytes + rec_bytes + side_bytes > EB_NOALLOC_SCRATCH_BYTES) return EB_ERR_OVERFLOW;
+  if (ebk::stream_layout<DT>(1).total > d.optin) return EB_ERR_OVERFLOW;
 
-  unsigned char* ctrl = d.scratch;
-  if (cudaMemsetAsync(ctrl, 0, kNoAllocCtrlBytes, st) != cudaSuccess) return EB_ERR_CUDA;
+  unsigned char* ctrl = nd.scratch;
+  Rec* recs = reinterpret_cast<Rec*>(nd.scratch + kNoAllocCtrlBytes);
+  int32_t* cnt = reinterpret_cast<int32_t*>(nd.scratch + kNoAllocCtrlBytes + rec_bytes);
+  float* pmax = reinterpret_cast<float*>(cnt + rows);
+  int32_t* sample = reinterpret_cast<int32_t*>(pmax + rows);
+  if (cudaMemsetAsync(ctrl, 0, kNoAllocCtrlBytes, st) != cudaSuccess ||
+      cudaMemsetAsync(cnt, 0, (size_t)rows * sizeof(int32_t), st) != cudaSuccess)
+    return EB_ERR_CUDA;
   StepArgs a;
   std::memset(&a, 0, sizeof(a));
   a.logits = logits;
   a.H_out = entropies;
   a.amax_out = argmax;
-  a.stop_flags = ctrl;                                         // one pseudo-canvas, active
+  a.stop_flags = ctrl;  // one pseudo-canvas, active
   a.status = reinterpret_cast<uint32_t*>(ctrl + 4);
   a.act_index = reinterpret_cast<int32_t*>(ctrl + 8);
   a.n_act = reinterpret_cast<int32_t*>(ctrl + 12);
-  a.partials = reinterpret_cast<Partial*>(d.scratch + kNoAllocCtrlBytes);
+  a.recs = recs;
+  a.row_cnt = cnt;
+  a.pmax = pmax;
+  a.sample = sample;
+  a.wait_ns = ebk::kWaitLimitNs;
   a.B = 1;
   a.L = rows;  // the rows are the positions of one pseudo-canvas
   a.V = V;
@@ -716,24 +730,21 @@ int noalloc_launch(const NoAllocDevice& d, const void* logits, int32_t rows, int
   a.s = 0;
   a.N = 1;
   a.max_segs = max_segs;
-  a.nw = nw;
   a.G1 = grid;
   const size_t elt = DT == ebk::kF32 ? 4 : 2;
   a.vec_ok = ((uintptr_t)logits % 16 == 0) && (((size_t)V * elt) % 16 == 0) ? 1 : 0;
   a.greedy = 1;  // no draw: the stream pass skips the Gumbel race
   a.c2 = (float)(1.4426950408889634 / T);
   a.iT = (float)(1.0 / T);
+  a.V_tot = V;
   void* args[] = {&a};
   if (cudaLaunchKernel(reinterpret_cast<const void*>(&ebk::stream_kernel<DT>), dim3(grid),
                        dim3(Sh::kThreads), args, ebk::stream_layout<DT>(1).total, st) !=
       cudaSuccess)
     return EB_ERR_CUDA;
-  const int32_t* n_act = a.n_act;
-  void* rargs[] = {&a, &n_act};
-  if (cudaLaunchKernel(reinterpret_cast<const void*>(&ebk::row_stats_kernel<DT>),
-                       dim3((unsigned)((rows + 31) / 32)), dim3(256), rargs, 0, st) !=
-      cudaSuccess)
-    return EB_ERR_CUDA;
+  ebk::noalloc_mark_kernel<<<std::min(64, (rows + 255) / 256), 256, 0, st>>>(a.status, entropies,
+                                                                             argmax, rows);
+  if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   return EB_OK;
 }
 
@@ -750,12 +761,16 @@ extern "C" int eb_row_stats_noalloc(const void* logits, int dtype, int32_t rows,
     return EB_ERR_OVERFLOW;
   int device = 0;
   if (cudaGetDevice(&device) != cudaSuccess) return EB_ERR_CUDA;
-  if (device < 0 || device >= kNoAllocMaxDevices) return EB_ERR_UNSUPPORTED;
-  NoAllocDevice& d = g_noalloc_dev[device];
-  std::call_once(d.once, noalloc_setup, std::ref(d), device);
-  if (d.rc != EB_OK) return d.rc;
+  DeviceAttrs* d = nullptr;
+  int rc = device_attrs(device, &d);
+  if (rc != EB_OK) return rc;
+  NoAllocDevice& nd = g_noalloc_dev[device];
+  std::call_once(nd.once, noalloc_setup, std::ref(nd));
+  if (nd.rc != EB_OK) return nd.rc;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   return dtype == EB_F32
-             ? noalloc_launch<ebk::kF32>(d, logits, rows, V, temperature, entropies, argmax, st)
-             : noalloc_launch<ebk::kBF16>(d, logits, rows, V, temperature, entropies, argmax, st);
+             ? noalloc_launch<ebk::kF32>(nd, *d, logits, rows, V, temperature, entropies, argmax,
+                                         st)
+             : noalloc_launch<ebk::kBF16>(nd, *d, logits, rows, V, temperature, entropies, argmax,
+                                          st);
 }

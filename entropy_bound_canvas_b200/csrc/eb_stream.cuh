@@ -1,26 +1,32 @@
 // eb_stream.cuh -- first kernel of a sampler step: one pass over every logit
-// of every active canvas.
+// of every active canvas, and each position's results.
 //
 // Work split.  The active rows' 64-logit groups are numbered g = row ng + j
 // (row = active canvas index * L + position).  Stream CTA c of G (one per SM)
 // owns the contiguous range [c NG / G, (c + 1) NG / G): every CTA reads the
 // same number of bytes to within one group, and a row meets only a few CTAs.
 //
-// Inside a CTA.  The producer warp walks the range in tiles of up to
-// kStageGroups groups that never straddle a row.  For each tile it writes the
-// tile's description and, for an open position, the group-stream Philox
-// words of the tile's groups into the stage's header in shared memory; lane 0
-// then copies the tile into a kStages-deep ring with one 1-D bulk copy (the
-// TMA engine, no multicast, L2 evict-first).  A tile is cut into sub-tiles of
-// 64 groups, dealt round-robin to the consumer warps (a fixed assignment, so
-// every run sums in the same order).  A lane reduces two groups of its warp's
-// sub-tile; the warp shares one running maximum per row (WarpAcc), so its
-// lanes' sums stay relative to the same reference and the Gumbel race runs
-// against the warp's best.  When a warp moves on to another row it sums its
-// lanes and writes one Partial record for (row, CTA, warp); it writes an
-// empty record for
-// each row of its CTA's range that it never touched, so the finish kernel
-// only ever reads records written during this step.
+// Inside a CTA (one CTA per SM):
+//   - the copy producer (one lane) walks the range in tiles of up to
+//     kStageGroups groups that never straddle a row, writes each tile's
+//     description and copies it into a kStages-deep ring with one 1-D bulk
+//     copy (the TMA engine, no multicast, L2 evict-first);
+//   - the word producer computes the group-stream Philox words of an open
+//     position's tiles;
+//   - twelve consumer warps take the tiles' 64-group sub-tiles round-robin
+//     (a fixed assignment, so every run sums in the same order).  A lane
+//     reduces two groups per sub-tile into its own running state (Acc): for
+//     bf16 logits it copies both groups into registers and releases the
+//     stage before any arithmetic, so the ring refills while it computes.
+//     When a warp leaves a row it merges its lanes and deposits one record
+//     per row of the CTA's range into a shared-memory slot;
+//   - the finisher warp merges the twelve deposits of each row into the
+//     CTA's record.  A row spread over several CTAs exchanges records through
+//     global memory: each CTA writes its record and counts itself in the
+//     row's counter; the last one merges them all (in CTA order) and
+//     finishes the row: entropy, max probability, argmax, and for an open
+//     position the element draw inside the winning Gumbel group.
+// The per-canvas decisions run in the epilogue kernel (eb_finish.cuh).
 #pragma once
 
 #include "eb_common.cuh"
@@ -36,40 +42,35 @@ namespace ebk {
 #ifndef EB_STREAM_STAGE_KB
 #define EB_STREAM_STAGE_KB 32
 #endif
-#ifndef EB_STREAM_GROUPS_PER_LANE
-#define EB_STREAM_GROUPS_PER_LANE 2
-#endif
 
 constexpr int kStages = EB_STREAM_STAGES;
+constexpr int kSlots = 8;  // row slots of the consumer -> finisher hand-off
 
-// Shape of the stream CTA: kConsumerWarps consumer warps + 2 producer warps,
-// a ring of kStages stages of kStageBytes each (192 KB with the defaults:
-// one CTA per SM).  Twelve consumer warps, each lane reducing two groups at
-// a time, keep the SM's MUFU and FMA pipes busy.
 template <int DT>
 struct StreamShape {
   static constexpr int kConsumerWarps = EB_STREAM_CONSUMER_WARPS;
-  static constexpr int kThreads = (kConsumerWarps + 2) * 32;  // + copy and word producers
+  // + copy producer, word producer, finisher
+  static constexpr int kThreads = (kConsumerWarps + 3) * 32;
   static constexpr int kStageBytes = EB_STREAM_STAGE_KB * 1024;
   // room for a copy widened to 16-byte boundaries; 128-byte aligned stages
   static constexpr int kStageStride = kStageBytes + 128;
   static constexpr int kStageGroups = kStageBytes / (kGroup * elt_bytes(DT));
-  static constexpr int kGroupsPerLane = EB_STREAM_GROUPS_PER_LANE;
-  static constexpr int kSubGroups = 32 * kGroupsPerLane;  // groups per sub-tile
+  static constexpr int kSubGroups = 64;  // groups per sub-tile: two per lane
   static constexpr int kSubPerStage = kStageGroups / kSubGroups;
   static_assert(kSubPerStage >= 1 && (kSubPerStage & (kSubPerStage - 1)) == 0,
                 "sub-tiles per stage must be a power of two");
+  static_assert(kConsumerWarps <= 16, "the finisher merges at most 16 deposits per row");
 };
 
 __host__ __device__ constexpr int stream_threads(int dt) {
   return dt == kBF16 ? StreamShape<kBF16>::kThreads : StreamShape<kF32>::kThreads;
 }
-__host__ __device__ constexpr int stream_consumer_warps() { return EB_STREAM_CONSUMER_WARPS; }
 
 struct StreamCtrl {
   int abort;
   int issued;  // tiles whose bulk copy has been issued
   int n_sub;   // sub-tiles of this CTA's range
+  int words_arrived;  // tiles whose second (header) arrival was made
   int wcnt[32];
 };
 
@@ -85,8 +86,16 @@ struct TileMeta {
   int pad;
 };
 
+// A row slot: the consumer warps' deposits for one row of the CTA's range.
+struct RowSlot {
+  int q;      // CTA-relative row the slot accepts deposits for
+  int count;  // deposits made
+  int pad0, pad1;
+  Acc rec[EB_STREAM_CONSUMER_WARPS];
+};
+
 struct StreamLayout {
-  uint32_t bars, ctrl, meta, words, act, ring, total;
+  uint32_t bars, ctrl, meta, words, slots, act, ring, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -104,6 +113,8 @@ __host__ __device__ inline StreamLayout stream_layout(int B) {
   o = align_up(o + (uint32_t)sizeof(TileMeta) * kStages, 16);
   y.words = o;
   o = align_up(o + 4u * (uint32_t)Sh::kStageGroups * kStages, 16);
+  y.slots = o;
+  o = align_up(o + (uint32_t)sizeof(RowSlot) * kSlots, 16);
   y.act = o;
   o = align_up(o + 2u * (uint32_t)B, 128);
   y.ring = o;
@@ -178,7 +189,7 @@ __device__ __forceinline__ int count_tiles(unsigned long long lo, unsigned long 
 }
 
 // Active canvases in index order, from the stop flags as they were when the
-// step began (only the finish kernel, after this one, writes them).
+// step began (only the epilogue kernel, after this one, writes them).
 __device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int B, uint16_t* act,
                                                  int* wcnt, int nthreads) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -199,11 +210,263 @@ __device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int 
   return base;
 }
 
+// Where row r's records live: the stream CTAs that own part of it are
+// c_first .. c_last; with at least one group per CTA (NG >= G) record `seg`
+// of CTA c is c - c_first, otherwise every CTA owns at most one group and
+// the record index is that group's index in the row.
+struct RowSpan {
+  int seg, nseg;
+};
+__device__ __forceinline__ RowSpan row_span(unsigned long long r, int ng, unsigned long long NG,
+                                            int G, int c) {
+  const unsigned long long g0 = r * (unsigned long long)ng;
+  RowSpan s;
+  if (NG >= (unsigned long long)G) {
+    const int c0 = cta_of(g0, NG, G);
+    const int c1 = cta_of(g0 + (unsigned long long)ng - 1ull, NG, G);
+    s.seg = c - c0;
+    s.nseg = c1 - c0 + 1;
+  } else {
+    s.seg = (int)(range_start(c, NG, G) - g0);
+    s.nseg = ng;
+  }
+  return s;
+}
+
+// ---------------------------------------------------------------------------
+// Finishing a row (one warp): the merged state of all its groups -> the
+// position's outputs.  Entropy and max probability in float64 from the
+// exact top-group count and the small sums; the element draw inside the
+// winning group reads that group's 64 logits and their element-stream
+// Philox words: the largest tempered logit is drawn first, and the
+// logarithms of every element that provably cannot beat it are skipped.
+// ---------------------------------------------------------------------------
+// The final combine of a row's n records, in stream-CTA order (which is
+// group order): the row maximum, the record holding its top group (the
+// first record attaining it), every record's sums rescaled to the maximum
+// in float64 -- except the top record's top-group sums, which the exact
+// recomputation replaces -- and the best Gumbel ratio (lower group on equal
+// ratios).  `rec(i)` loads record i; every lane returns the same values.
+struct RowFinal {
+  double S, W;  // relative to M, W in log2 units, without the top group
+  float M;
+  int tj;       // top group (local id; kNone: no finite logit)
+  float R;      // best ratio relative to M
+  int gb;       // its group (kNone: none)
+};
+
+template <class Load>
+__device__ __forceinline__ RowFinal combine_records(int n, Load rec, float c2) {
+  float M = -INFINITY;
+  for (int i = threadIdx.x & 31; i < n; i += 32) M = fmaxf(M, rec(i).M);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  // the top record: the first whose maximum is M
+  int top = kNone;
+  for (int i = threadIdx.x & 31; i < n; i += 32)
+    if (rec(i).M == M && M > -INFINITY) top = min(top, i);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) top = min(top, __shfl_xor_sync(0xffffffffu, top, o));
+  double S = 0.0, W = 0.0;
+  float Rl = 0.f;
+  int gl = kNone, tj = kNone;
+  for (int i = threadIdx.x & 31; i < n; i += 32) {
+    const Acc c = rec(i);
+    if (!(c.M > -INFINITY)) continue;
+    const bool tie = c.M == M;
+    const double dd = tie ? 0.0 : (double)((c.M - M) * c2);
+    const double f = tie ? 1.0 : exp2(dd);
+    double So = (double)c.Sr, Wo = (double)c.Wr;
+    if (i == top) {
+      tj = c.tj;
+    } else {
+      So += (double)c.tS;
+      Wo += (double)c.tW;
+    }
+    S += f * So;
+    W += f * (Wo + dd * So);
+    const float Rc = c.R * (float)f;
+    if (Rc > Rl || (Rc == Rl && Rc > 0.f && c.gb < gl)) {
+      Rl = Rc;
+      gl = c.gb;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    S += __shfl_xor_sync(0xffffffffu, S, o);
+    W += __shfl_xor_sync(0xffffffffu, W, o);
+    const float oR = __shfl_xor_sync(0xffffffffu, Rl, o);
+    const int og = __shfl_xor_sync(0xffffffffu, gl, o);
+    if (oR > Rl || (oR == Rl && oR > 0.f && og < gl)) {
+      Rl = oR;
+      gl = og;
+    }
+    tj = min(tj, __shfl_xor_sync(0xffffffffu, tj, o));
+  }
+  RowFinal f;
+  f.S = S;
+  f.W = W;
+  f.M = M;
+  f.tj = tj;
+  f.R = Rl;
+  f.gb = gl;
+  return f;
+}
+
+// This lane's two elements 2 lane, 2 lane + 1 of group j of a row (local
+// ids; those at or beyond V read as -inf).
+template <int DT>
+__device__ __forceinline__ float2 load_pair(const StepArgs& a, const char* rowp, int j) {
+  const int v0 = j * kGroup + 2 * (threadIdx.x & 31);
+  float2 z = make_float2(-INFINITY, -INFINITY);
+  if (a.vec_ok && v0 + 1 < a.V) {
+    if (DT == kF32) {
+      z = __ldg(reinterpret_cast<const float2*>(rowp) + (v0 >> 1));
+    } else {
+      const uint32_t w = __ldg(reinterpret_cast<const uint32_t*>(rowp) + (v0 >> 1));
+      z = make_float2(bf16_lo(w), bf16_hi(w));
+    }
+  } else {
+    if (v0 < a.V) z.x = load_elem<DT>(rowp, v0);
+    if (v0 + 1 < a.V) z.y = load_elem<DT>(rowp, v0 + 1);
+  }
+  return z;
+}
+
+// Element draw inside group j (local group id), whose elements this lane
+// holds as (z.x, z.y) = elements 2 lane, 2 lane + 1.  Every lane returns the
+// drawn local id (kNone if the group holds no finite logit).  The largest
+// tempered logit is drawn first, and the logarithms of every element that
+// provably cannot beat it are skipped.
+__device__ __forceinline__ int draw_in_group(const StepArgs& a, float2 z, int j, int bi, int l) {
+  const int lane = threadIdx.x & 31;
+  const int v0 = j * kGroup + 2 * lane;
+  // element-stream words: lane k < 16 computes call k of the group (global
+  // ids: the group starts on a multiple of 64, so on a call boundary)
+  const uint32_t gv0 = (uint32_t)(a.v_off + j * kGroup);
+  Words4 w4{{0u, 0u, 0u, 0u}};
+  if (lane < 16)
+    w4 = philox((gv0 >> 2) + (uint32_t)lane, (uint32_t)l, (uint32_t)a.s,
+                (uint32_t)(a.canvas_offset + bi) | (kStreamGumbel << 24), a.key0, a.key1);
+  const int src = lane >> 1;
+  const uint32_t s0 = __shfl_sync(0xffffffffu, w4.w[0], src);
+  const uint32_t s1 = __shfl_sync(0xffffffffu, w4.w[1], src);
+  const uint32_t s2 = __shfl_sync(0xffffffffu, w4.w[2], src);
+  const uint32_t s3 = __shfl_sync(0xffffffffu, w4.w[3], src);
+  const uint32_t x0 = (lane & 1) ? s2 : s0, x1 = (lane & 1) ? s3 : s1;
+  const float y0 = z.x * a.iT, y1 = z.y * a.iT;
+  float ym = y0;
+  int vm = v0;
+  uint32_t xm = x0;
+  if (y1 > ym) {
+    ym = y1;
+    vm = v0 + 1;
+    xm = x1;
+  }
+  if (!(ym > -INFINITY)) vm = kNone;
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float oy = __shfl_xor_sync(0xffffffffu, ym, o);
+    const int ov = __shfl_xor_sync(0xffffffffu, vm, o);
+    const uint32_t ox = __shfl_xor_sync(0xffffffffu, xm, o);
+    if (oy > ym || (oy == ym && ov < vm)) {
+      ym = oy;
+      vm = ov;
+      xm = ox;
+    }
+  }
+  if (vm == kNone) return kNone;
+  const float seed = ym + gumbel(xm);
+  float best = seed;
+  int barg = vm;
+  auto consider = [&](float y, int v, uint32_t x) {
+    if (v == vm || !(y > -INFINITY)) return;
+    // can v beat the seed?  It needs g > seed - y, i.e. -ln u < e^-(seed - y);
+    // -ln u >= 1 - u, so 1 - u >= e^-(seed - y) (1e-4 relative margin) rules it out.
+    const float tgap = seed - y;
+    if (tgap > -2.0f && one_minus_u(x) >= ex2(-1.4426950408889634f * tgap) * 1.0001f) return;
+    const float sc = y + gumbel(x);
+    if (sc > best || (sc == best && v < barg)) {
+      best = sc;
+      barg = v;
+    }
+  };
+  consider(y0, v0, x0);
+  consider(y1, v0 + 1, x1);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    const float ob = __shfl_xor_sync(0xffffffffu, best, o);
+    const int oa = __shfl_xor_sync(0xffffffffu, barg, o);
+    if (ob > best || (ob == best && oa < barg)) {
+      best = ob;
+      barg = oa;
+    }
+  }
+  return barg;
+}
+
+// Finishes row (bi, l) from the combined records (one warp): the exact form
+// of the top group (elements equal to the row maximum count 1 each, the
+// smaller ones are summed with d = (z - M) c2 from the exact difference)
+// gives, with the other sums, the entropy and max probability in float64
+// and the argmax; an open position draws inside the winning group.  Writes
+// the position's outputs (or, for a vocabulary slice, its slice record).
+template <int DT>
+__device__ __forceinline__ void finish_position(const StepArgs& a, const RowFinal& F, int bi, int l,
+                                                bool open) {
+  const int lane = threadIdx.x & 31;
+  const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
+  const char* rowp =
+      reinterpret_cast<const char*>(a.logits) + grow * (size_t)a.V * (size_t)elt_bytes(DT);
+  const bool draw = open && !a.greedy && F.gb != kNone;
+  // both groups' loads in flight together
+  float2 zt = make_float2(-INFINITY, -INFINITY), zd = zt;
+  if (F.tj != kNone) zt = load_pair<DT>(a, rowp, F.tj);
+  if (draw) zd = load_pair<DT>(a, rowp, F.gb);
+  Exact e{0.f, 0.f, 0, kNone};
+  if (F.tj != kNone) {
+    exact_elem(zt.x, F.tj * kGroup + 2 * lane, F.M, a.c2, e);
+    exact_elem(zt.y, F.tj * kGroup + 2 * lane + 1, F.M, a.c2, e);
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    e.S += __shfl_xor_sync(0xffffffffu, e.S, o);
+    e.W += __shfl_xor_sync(0xffffffffu, e.W, o);
+    e.n += __shfl_xor_sync(0xffffffffu, e.n, o);
+    e.amin = min(e.amin, __shfl_xor_sync(0xffffffffu, e.amin, o));
+  }
+  int x = kNone;
+  if (draw) x = draw_in_group(a, zd, F.gb, bi, l);
+  if (lane != 0) return;
+  const double S = (double)e.n + ((double)e.S + F.S);
+  const double W = (double)e.W + F.W;
+  const bool bad = !isfinite(S) || !isfinite(W) || F.tj == kNone || e.amin == kNone;
+  if (bad) atomicOr(a.status, kStatusNonFinite);
+  const int amax = e.amin == kNone ? kNone : e.amin + a.v_off;
+  const int smp = x == kNone ? kNone : x + a.v_off;
+  if (a.slice_out != nullptr) {
+    SliceRecord r;
+    r.S = S;
+    r.W = W;
+    r.zmax = F.M;
+    r.gscore = (F.R > 0.f && F.gb != kNone) ? fmaf(F.M, a.iT, logf(F.R)) : -INFINITY;
+    r.amax = amax;
+    r.sample = draw ? smp : -1;
+    r.pad0 = r.pad1 = 0;
+    a.slice_out[grow] = r;
+    return;
+  }
+  a.H_out[grow] = (float)(log(S) - 0.6931471805599453 * (W / S));
+  a.amax_out[grow] = amax;
+  a.pmax[grow] = (float)(1.0 / S);
+  a.sample[grow] = open ? (draw ? smp : amax) : -1;
+}
+
 // One CTA per SM: the register cap is the register file over the block.
 template <int DT>
 __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(const StepArgs a) {
   using Sh = StreamShape<DT>;
-  using IO = GroupIO<DT>;
+  constexpr int NW = Sh::kConsumerWarps;
   extern __shared__ __align__(128) unsigned char smem[];
   const StreamLayout lay = stream_layout<DT>(a.B);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
@@ -211,6 +474,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(smem + lay.ctrl);
   TileMeta* meta = reinterpret_cast<TileMeta*>(smem + lay.meta);
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + lay.words);
+  RowSlot* slots = reinterpret_cast<RowSlot*>(smem + lay.slots);
   uint16_t* act = reinterpret_cast<uint16_t*>(smem + lay.act);
   unsigned char* ring = smem + lay.ring;
 
@@ -222,10 +486,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     }
     ctrl->abort = 0;
     ctrl->issued = 0;
+    ctrl->words_arrived = 0;
+    for (int i = 0; i < kSlots; ++i) {
+      slots[i].q = i;
+      slots[i].count = 0;
+    }
     fence_mbar_init();
   }
   const int n_act = build_active_list(a.stop_flags, a.B, act, ctrl->wcnt, Sh::kThreads);
-  if (blockIdx.x == 0) {  // publish the active list for the finish kernel
+  if (blockIdx.x == 0) {  // publish the active list for the epilogue kernel
     for (int b = tid; b < a.B; b += Sh::kThreads) a.act_index[b] = -1;
     __syncthreads();
     for (int i = tid; i < n_act; i += Sh::kThreads) a.act_index[act[i]] = i;
@@ -238,18 +507,21 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   const unsigned long long g_hi = range_start(blockIdx.x + 1, NG, G);
   if (tid == 0) ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
   __syncthreads();
-  // The finish kernel may be scheduled from now on, wherever an SM has room:
-  // its CTAs load what the previous step left and then wait for this grid's
-  // completion (griddepcontrol.wait) before reading anything it writes.
+  // The epilogue kernel may be scheduled from now on, wherever an SM has
+  // room: its CTAs load what the previous step left and then wait for this
+  // grid's completion (griddepcontrol.wait) before reading anything it writes.
   griddep_launch_dependents();
 
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
   const char* logits = reinterpret_cast<const char*>(a.logits);
+  const long long r_first = (long long)(g_lo / (unsigned long long)a.ng);
+  const long long r_end =
+      g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
 
-  if (warp == Sh::kConsumerWarps) {
+  if (warp == NW) {
     // ------------------------------------------------------- copy producer
-    // Lane 0 alone: waits for a free stage, writes the tile's description
-    // and issues its bulk copy (the stage's first arrival, with the bytes).
+    // Lane 0 alone: waits for a free stage, issues the tile's bulk copy (the
+    // stage's first arrival, with the bytes) and writes its description.
     if (lane == 0) {
       const uint64_t policy = evict_first_policy();
       TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kStageGroups);
@@ -259,7 +531,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       long long row_seen = -1;
       int bi = 0, samp = 0;
       while (it.next(t)) {
-        if (k >= kStages && !mbar_wait(&empty[st], ph ^ 1u)) {
+        if (k >= kStages && !mbar_wait(&empty[st], ph ^ 1u, a.wait_ns)) {
           atomicOr(a.status, kStatusTimeout);
           *(volatile int*)&ctrl->abort = 1;
           break;
@@ -284,9 +556,6 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
                   (uint32_t)(a1 - a0), &full[st], policy);
         // The position's committed flag is read while the copy is in flight.
-        // Nothing reads the description before the release of `issued`, and
-        // the stage cannot fill before the word producer's arrival, which
-        // follows that release.
         if (new_row)
           samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
         TileMeta m;
@@ -307,17 +576,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         }
       }
     }
-  } else if (warp == Sh::kConsumerWarps + 1) {
+  } else if (warp == NW + 1) {
     // ------------------------------------------------------- word producer
-    // Follows the copy producer: once tile k is issued (so its stage is free
-    // and its description written), computes the group-stream Philox words
-    // of an open position's groups into the stage's header and makes the
-    // stage's second arrival.  Kept off the copy producer so that copies are
-    // never issued late.
+    // Once tile k is issued (its stage free and its description written),
+    // computes the group-stream Philox words of an open position's groups
+    // into the stage's header and makes the stage's second arrival.
     const int n_tiles = ctrl->n_sub / Sh::kSubPerStage;
     int st = 0, words_done = 0;
     for (int k = 0; k < n_tiles; ++k, words_done = k) {
-      if (!wait_counter_above(&ctrl->issued, k)) {
+      if (!wait_counter_above(&ctrl->issued, k, a.wait_ns)) {
         if (lane == 0) {
           atomicOr(a.status, kStatusTimeout);
           *(volatile int*)&ctrl->abort = 1;
@@ -343,50 +610,133 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       if (lane == 0) mbar_arrive(&full[st]);  // header (words) complete
       if (++st == kStages) st = 0;
     }
-    // After an abort: the second arrival of every tile already issued, so
-    // that the drain below sees each copy complete.
-    if (lane == 0 && *(volatile int*)&ctrl->abort) {
-      const int issued = ld_acquire_shared(&ctrl->issued);
-      for (int k = words_done; k < issued; ++k) mbar_arrive(&full[k % kStages]);
+    if (lane == 0) ctrl->words_arrived = words_done;
+  } else if (warp == NW + 2) {
+    // ------------------------------------------------------------ finisher
+    const int nrows = (int)(r_end - r_first);
+    for (int q = 0; q < nrows; ++q) {
+      RowSlot* sl = &slots[q % kSlots];
+      const long long r = r_first + q;
+      const int ai = (int)(r / a.L);
+      const int l = (int)(r - (long long)ai * a.L);
+      const int bi = act[ai];
+      const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
+      const bool open = a.committed != nullptr && a.committed[grow] == 0;
+      // the twelve deposits of row q
+      bool ok = true;
+      {
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_shared(&sl->count) < NW) {
+          if (*(volatile int*)&ctrl->abort || global_ns() - t0 > a.wait_ns) {
+            ok = false;
+            break;
+          }
+          __nanosleep(32);
+        }
+      }
+      if (!__all_sync(0xffffffffu, ok)) {
+        if (lane == 0) {
+          atomicOr(a.status, kStatusTimeout);
+          *(volatile int*)&ctrl->abort = 1;
+        }
+        break;
+      }
+      Acc mine;
+      if (lane < NW) {
+        mine = sl->rec[lane];
+      } else {
+        acc_reset(mine);
+      }
+      warp_merge_acc(mine, a.c2, 16);
+      __syncwarp();
+      if (lane == 0) {
+        sl->count = 0;
+        st_release_shared(&sl->q, q + kSlots);
+      }
+      // the row's other stream CTAs
+      const RowSpan sp = row_span((unsigned long long)r, a.ng, NG, G, blockIdx.x);
+      if (sp.nseg == 1) {
+        // lanes below 16 hold the CTA's merged state
+        const RowFinal F = combine_records(1, [&](int) { return mine; }, a.c2);
+        finish_position<DT>(a, F, bi, l, open);
+        continue;
+      }
+      Rec* rr = a.recs + grow * (size_t)a.max_segs;
+      int last = 0;
+      if (lane == 0) {
+        Rec w;
+        w.a = mine;
+        rr[sp.seg] = w;
+        __threadfence();
+        last = atomicAdd(a.row_cnt + grow, 1) == sp.nseg - 1;
+      }
+      last = __shfl_sync(0xffffffffu, last, 0);
+      if (!last) continue;
+      __threadfence();
+      auto load = [&](int i) {
+        const Acc* p = &rr[i].a;
+        Acc c;
+        c.M = __ldcg(&p->M);
+        c.tS = __ldcg(&p->tS);
+        c.tW = __ldcg(&p->tW);
+        c.Sr = __ldcg(&p->Sr);
+        c.Wr = __ldcg(&p->Wr);
+        c.R = __ldcg(&p->R);
+        c.tj = __ldcg(&p->tj);
+        c.gb = __ldcg(&p->gb);
+        return c;
+      };
+      const RowFinal F = combine_records(sp.nseg, load, a.c2);
+      if (lane == 0) a.row_cnt[grow] = 0;  // zero again for the next step
+      finish_position<DT>(a, F, bi, l, open);
     }
   } else {
     // ------------------------------------------------------------ consumers
     const int n_sub = ctrl->n_sub;
-    const long long r_first = (long long)(g_lo / (unsigned long long)a.ng);
-    const long long r_end =
-        g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
-    // slot of this CTA among the CTAs of its first row; later rows start in it
-    const int seg_first =
-        (int)blockIdx.x - cta_of((unsigned long long)r_first * (unsigned long long)a.ng, NG, G);
-    const size_t spr = (size_t)(a.max_segs * a.nw);
-    auto record_of = [&](long long r, int bi, int l) {
-      const int seg = r == r_first ? seg_first : 0;
-      return ((size_t)bi * (size_t)a.L + (size_t)l) * spr + (size_t)(seg * a.nw + warp);
-    };
     long long cur_r = -1;
-    long long next_r = r_first;  // first row of the range this warp still owes a record
-    size_t cur_rec = 0;
+    long long next_r = r_first;  // first row of the range this warp still owes a deposit
     int sampling = 0;
-    WarpAcc A;
-    warp_reset(A);
+    Acc A;
+    acc_reset(A);
     const int rot = lane;
+    bool fail = false;
 
-    auto owe_empty = [&](long long upto) {
-      for (; next_r < upto; ++next_r) {
-        if (lane == 0) {
-          const int ai = (int)(next_r / a.L);
-          const int l = (int)(next_r - (long long)ai * a.L);
-          a.partials[record_of(next_r, act[ai], l)] = empty_partial();
+    // This warp's record of CTA-relative row q into its slot (after the
+    // finisher has released the slot's previous row).
+    auto deposit = [&](long long r, bool empty_rec) -> bool {
+      Acc w = A;
+      if (!empty_rec) warp_merge_acc(w, a.c2);
+      const int q = (int)(r - r_first);
+      RowSlot* sl = &slots[q % kSlots];
+      int ok = 1;
+      if (lane == 0) {
+        const uint64_t t0 = global_ns();
+        while (ld_acquire_shared(&sl->q) != q) {
+          if (*(volatile int*)&ctrl->abort || global_ns() - t0 > a.wait_ns) {
+            ok = 0;
+            break;
+          }
+          __nanosleep(32);
+        }
+        if (ok) {
+          if (empty_rec) {
+            sl->rec[warp].M = -INFINITY;
+          } else {
+            sl->rec[warp] = w;
+          }
+          red_release_shared_add(&sl->count, 1);
         }
       }
+      return __shfl_sync(0xffffffffu, ok, 0) != 0;
     };
-    auto flush = [&]() {
-      const Partial P = warp_record(A, a.iT);
-      if (lane == 0) a.partials[cur_rec] = P;
+    auto owe_empty = [&](long long upto) -> bool {
+      for (; next_r < upto; ++next_r)
+        if (!deposit(next_r, true)) return false;
+      return true;
     };
 
-    // Sub-tiles are dealt round-robin: warp w takes w, w + nw, w + 2 nw, ...
-    for (int u = warp; u < n_sub; u += Sh::kConsumerWarps) {
+    // Sub-tiles are dealt round-robin: warp w takes w, w + NW, w + 2 NW, ...
+    for (int u = warp; u < n_sub; u += NW) {
       if (*(volatile int*)&ctrl->abort) break;
       const int k = u / Sh::kSubPerStage;
       const int sub = u & (Sh::kSubPerStage - 1);
@@ -394,102 +744,136 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       // A warp may run up to a few sub-tiles ahead of the ring, past the
       // stage's current phase; the parity of the full barrier is only
       // unambiguous once the producer has issued tile k (which it does after
-      // the stage's previous tile, k - kStages, was released).
-      if (!wait_counter_above(&ctrl->issued, k) ||
-          !mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u)) {
-        if (lane == 0) {
-          atomicOr(a.status, kStatusTimeout);
-          *(volatile int*)&ctrl->abort = 1;
-        }
+      // the stage's previous tile, k - kStages, was released).  The row
+      // change (and its deposits) is handled before the stage is waited for,
+      // so a warp never holds a stage while it waits for a row slot.
+      if (!wait_counter_above(&ctrl->issued, k, a.wait_ns)) {
+        fail = true;
         break;
       }
       const TileMeta m = meta[st];
       if (m.r != cur_r) {
-        if (cur_r >= 0) flush();
-        owe_empty(m.r);
+        if (cur_r >= 0 && !deposit(cur_r, false)) {
+          fail = true;
+          break;
+        }
+        if (cur_r >= 0) next_r = cur_r + 1;
+        if (!owe_empty(m.r)) {
+          fail = true;
+          break;
+        }
         cur_r = m.r;
         next_r = cur_r + 1;
-        cur_rec = record_of(cur_r, m.bi, m.l);
         sampling = m.sampling;
-        warp_reset(A);
+        acc_reset(A);
+      }
+      if (!mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u, a.wait_ns)) {
+        fail = true;
+        break;
       }
       const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
-      if (sub * Sh::kSubGroups < m.cnt) {  // warp-uniform
-        const bool has0 = gl0 < m.cnt, has1 = Sh::kGroupsPerLane == 2 && gl1 < m.cnt;
-        const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
-        const unsigned char* gp0 = sbase + (size_t)(has0 ? gl0 : 0) * kGroup * elt_bytes(DT);
-        const unsigned char* gp1 = has1 ? sbase + (size_t)gl1 * kGroup * elt_bytes(DT) : gp0;
-        const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
-        const int len0 = has0 ? min(kGroup, a.V - j0 * kGroup) : 0;
-        const int len1 = has1 ? min(kGroup, a.V - j1 * kGroup) : 0;
-        const bool fast = a.vec_ok && (!has0 || len0 == kGroup) && (!has1 || len1 == kGroup);
-        float mg0, mg1;
-        if (fast) {
-          mg0 = IO::max_of(gp0, rot);
-          mg1 = Sh::kGroupsPerLane == 2 ? IO::max_of(gp1, rot) : -INFINITY;
+      const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
+      const uint32_t* wd = words + st * Sh::kStageGroups;
+      const bool any = sub * Sh::kSubGroups < m.cnt;  // warp-uniform
+      const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
+      const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
+      const int len0 = has0 ? min(kGroup, a.V - j0 * kGroup) : 0;
+      const int len1 = has1 ? min(kGroup, a.V - j1 * kGroup) : 0;
+      // whole 16-byte-aligned groups (or none) in every lane: the vector path
+      const bool fast =
+          __all_sync(0xffffffffu, a.vec_ok && (!has0 || len0 == kGroup) && (!has1 || len1 == kGroup));
+      uint32_t x0 = 0, x1 = 0;
+      if (sampling) {
+        if (has0) x0 = wd[gl0];
+        if (has1) x1 = wd[gl1];
+      }
+      // The lane's step for group j with maximum mg: a new maximum makes it
+      // the lane's top group (exact form); otherwise its sums join the rest
+      // (term by term when the vector sums are not finite: -inf logits).
+      // The lane's step for group j with maximum mg: a new maximum makes it
+      // the lane's top group; otherwise its sums join the rest.
+      // sums(ref, S, W): the group's sums relative to ref.
+      auto fold = [&](float mg, int j, uint32_t x, auto sums) {
+        if (!(mg > -INFINITY)) return;  // every logit -inf: nothing, never drawn
+        const bool new_top = mg > A.M;
+        float S, W;
+        sums(new_top ? mg : A.M, S, W);
+        float Z;
+        if (new_top) {
+          Z = lane_new_top(A, mg, j, S, W, a.c2);
         } else {
-          mg0 = has0 ? group_max_safe<DT>(gp0, len0) : -INFINITY;
-          mg1 = has1 ? group_max_safe<DT>(gp1, len1) : -INFINITY;
+          A.Sr += S;
+          A.Wr += W;
+          Z = S;
         }
-        if (!has0) mg0 = -INFINITY;
-        if (!has1) mg1 = -INFINITY;
-        warp_raise(A, fmaxf(mg0, mg1), mg0 >= mg1 ? j0 : j1, a.c2);
-        float S0 = 0.f, W0 = 0.f, S1 = 0.f, W1 = 0.f;
-        if (fast) {
-          if constexpr (Sh::kGroupsPerLane == 2) {
-            IO::exp2_of(gp0, gp1, rot, a.c2, A.M, A.M, S0, W0, S1, W1);
-          } else {
-            IO::exp1_of(gp0, rot, a.c2, A.M, S0, W0);
-          }
-          // -inf (or other non-finite) logits: redo the group term by term
-          if (!(W0 >= -3.0e38f)) {
-            const float2 q = group_sums_safe<DT>(gp0, kGroup, a.c2, A.M);
-            S0 = q.x;
-            W0 = q.y;
-          }
-          if (has1 && !(W1 >= -3.0e38f)) {
-            const float2 q = group_sums_safe<DT>(gp1, kGroup, a.c2, A.M);
-            S1 = q.x;
-            W1 = q.y;
-          }
-        } else {
-          if (has0) {
-            const float2 q = group_sums_safe<DT>(gp0, len0, a.c2, A.M);
-            S0 = q.x;
-            W0 = q.y;
-          }
-          if (has1) {
-            const float2 q = group_sums_safe<DT>(gp1, len1, a.c2, A.M);
-            S1 = q.x;
-            W1 = q.y;
-          }
-        }
-        if (has0) warp_fold(A, S0, W0, j0);
-        if (has1) warp_fold(A, S1, W1, j1);
-        if (sampling) {
-          const uint32_t* wd = words + st * Sh::kStageGroups;
-          float Rl = A.R;
-          int gbl = 0x7fffffff;
-          if (has0) lane_race(Rl, gbl, S0, wd[gl0], j0);
-          if (has1) lane_race(Rl, gbl, S1, wd[gl1], j1);
-          warp_race_merge(A, Rl, gbl);
-        }
+        if (sampling) lane_race(A, Z, x, j);
+      };
+      if (DT == kBF16 && fast && any) {
+        // both groups into registers, then the stage goes back to the producer
+        uint32_t G0[32], G1[32];
+        load_group_bf16(sbase + (size_t)(has0 ? gl0 : 0) * 128, rot, G0);
+        load_group_bf16(sbase + (size_t)(has1 ? gl1 : has0 ? gl0 : 0) * 128, rot, G1);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
+        if (has0)
+          fold(group_max_bf16(G0), j0, x0, [&](float ref, float& S, float& W) {
+            group_sums_bf16(G0, a.c2, ref, S, W);
+            if (!(W >= -3.0e38f && S <= 3.0e38f)) group_sums_bf16<true>(G0, a.c2, ref, S, W);
+          });
+        if (has1)
+          fold(group_max_bf16(G1), j1, x1, [&](float ref, float& S, float& W) {
+            group_sums_bf16(G1, a.c2, ref, S, W);
+            if (!(W >= -3.0e38f && S <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S, W);
+          });
+        continue;
+      }
+      if (any) {
+        auto group = [&](bool has, int gl, int len, int j, uint32_t x) {
+          if (!has) return;
+          const unsigned char* gp = sbase + (size_t)gl * kGroup * elt_bytes(DT);
+          const bool vec = DT == kF32 && fast;
+          fold(vec ? group_max_f32(gp, rot) : elem_max<DT>(gp, len), j, x,
+               [&](float ref, float& S, float& W) {
+                 if (vec) {
+                   group_sums_f32(gp, rot, a.c2, ref, S, W);
+                   if (W >= -3.0e38f && S <= 3.0e38f) return;
+                 }
+                 const Exact e = elem_exact<DT>(gp, len, ref, a.c2);  // term by term
+                 S = (float)e.n + e.S;
+                 W = e.W;
+               });
+        };
+        group(has0, gl0, len0, j0, x0);
+        group(has1, gl1, len1, j1, x1);
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
-    if (cur_r >= 0) flush();
-    owe_empty(r_end);
+    if (!fail && !*(volatile int*)&ctrl->abort) {
+      if (cur_r >= 0) {
+        if (!deposit(cur_r, false)) fail = true;
+        next_r = cur_r + 1;
+      }
+      if (!fail && !owe_empty(r_end)) fail = true;
+    }
+    if (fail && lane == 0) {
+      atomicOr(a.status, kStatusTimeout);
+      *(volatile int*)&ctrl->abort = 1;
+    }
   }
 
   __syncthreads();
   // After an abort, wait (bounded) for bulk copies still in flight into this
-  // CTA's shared memory before it may exit.
+  // CTA's shared memory before it may exit.  Every role has left its loop, so
+  // the issued count is final: first make the second arrival of every issued
+  // tile the word producer did not reach, so each stage's last phase can
+  // complete once its copy lands.
   if (tid == 0 && *(volatile int*)&ctrl->abort) {
     const int issued = ld_acquire_shared(&ctrl->issued);
+    for (int k = ctrl->words_arrived; k < issued; ++k) mbar_arrive(&full[k % kStages]);
     for (int st = 0; st < kStages && st < issued; ++st) {
       const int n2 = (issued - st + kStages - 1) / kStages;
-      mbar_wait(&full[st], (uint32_t)(n2 - 1) & 1u);
+      mbar_wait(&full[st], (uint32_t)(n2 - 1) & 1u, kDrainLimitNs);
     }
   }
 }

@@ -135,10 +135,12 @@ typedef struct {
 void eb_config_default(eb_config_t* cfg, int32_t B, int32_t L, int32_t V);
 
 /* Create a sampler on CUDA device `device` (the device must be sm_100).
-   Validates cfg, allocates and zeroes the workspace (the per-position
-   partial records of the stream pass, the active-canvas list, previous
-   argmax, stability counters, per-position draws and max probabilities,
-   status word) in one allocation.
+   Validates cfg, allocates and zeroes the workspace (the per-(position,
+   stream CTA) records and per-position counters of the stream pass, the
+   active-canvas list, previous argmax, stability counters, per-position
+   draws and max probabilities, status word) in one allocation.  The first
+   handle on a device also sets the kernels' shared-memory attributes for
+   that device (once, to the device maximum).
    On success *out owns the handle (release with eb_sampler_destroy).
    Errors: INVALID_ARG, OVERFLOW, UNSUPPORTED, OUT_OF_MEMORY, CUDA. */
 int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device);
@@ -192,29 +194,35 @@ int eb_sampler_set_state(eb_sampler_t* h, const int32_t* prev_argmax, const int3
    `entropies` ([rows] fp32, device) and its argmax (lowest index on ties)
    into `argmax` ([rows] int32, device), enqueued on `stream`.  These are the
    entropies and argmax that eb_sampler_step computes for a position at the
-   same temperature (bit for bit when the sampler's L lies in 129 .. 256, so
-   that both use the same per-position lane count).
+   same temperature (bit for bit against a one-canvas sampler with L = rows,
+   which splits the work across the GPU the same way).
 
    For callers that cannot allocate device memory, or must not: code that
    runs under a hard device-memory budget, a plugin handed raw pointers by a
    host that owns the allocator, or a caller that has no eb_sampler_t
    (eb_sampler_init allocates its workspace).  This call allocates nothing:
-   its scratch (the per-(row, SM, warp) partial records of the stream pass)
-   is a static device array of EB_NOALLOC_SCRATCH_BYTES bytes in the
-   library, looked up once per device.
-     - The first call on a device performs that one-time setup (symbol
-       lookup, kernel attributes); make it before any stream capture.
-     - Sizes beyond the scratch return EB_ERR_OVERFLOW: rows x (stream CTAs
-       a row can span) x 12 records x 32 bytes must fit (e.g. up to 8192
-       rows of 262144 logits).
-     - Calls that overlap in time (different streams or threads) share the
-       scratch and race; serialise them.
-   Non-finite softmax sums set bit EB_STATUS_NONFINITE of the scratch status
-   word, which is cleared at the start of every call and not otherwise
-   reported.  Returns EB_ERR_INVALID_ARG for NULL pointers, rows or V < 1, a
-   temperature that is not finite and positive, or logits not aligned to
-   their element size.  No counterpart in the DiffusionGemma pages: it
-   exposes the sampler's row reduction on its own, for deployment. */
+   its scratch (the stream pass's per-(row, stream CTA) records, per-row
+   counters and side outputs) is a static device array of
+   EB_NOALLOC_SCRATCH_BYTES bytes in the library, which every GPU that loads
+   the library holds until the process exits.
+     - The first call on a device performs a one-time setup on it (the
+       scratch's device address, kernel attributes); make it before any
+       stream capture.
+     - Sizes beyond the scratch return EB_ERR_OVERFLOW: 256 + rows x (48 x
+       the stream CTAs a row can span + 12) bytes must fit (about 50000 rows
+       of 262144 logits).
+     - Every call clears what must start at zero; calls that overlap in time
+       (different streams or threads) share the scratch and race: serialise
+       them.
+   If an internal wait of the pass gives up (EB_STATUS_TIMEOUT in the
+   scratch status word), every row's entropy is written as NaN and its
+   argmax as -1 instead of being left stale.  Non-finite softmax sums set
+   EB_STATUS_NONFINITE in that word, which is cleared at the start of every
+   call and not otherwise reported.  Returns EB_ERR_INVALID_ARG for NULL
+   pointers, rows or V < 1, a temperature that is not finite and positive,
+   or logits not aligned to their element size.  No counterpart in the
+   DiffusionGemma pages: it exposes the sampler's row reduction on its own,
+   for deployment. */
 #define EB_NOALLOC_SCRATCH_BYTES (8u << 20)
 int eb_row_stats_noalloc(const void* logits, int dtype, int32_t rows, int32_t V,
                          double temperature, float* entropies, int32_t* argmax, void* stream);
@@ -254,12 +262,25 @@ size_t eb_slice_record_bytes(void);
 
 /* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
    the caller) is non-NULL, every following eb_sampler_step records it on
-   its stream between the step's two kernels, so that the caller can time
-   them apart with events recorded before and after the call.  Recording it
-   keeps the second kernel from starting early (programmatic dependent
-   launch), so set it only for timing; NULL turns it off.  No counterpart in
-   the method: it measures the implementation. */
+   its stream between the step's two kernels (the stream pass and the canvas
+   epilogue), so that the caller can time them apart with events recorded
+   before and after the call.  Recording it keeps the second kernel from
+   starting early (programmatic dependent launch), so set it only for
+   timing; NULL turns it off.  No counterpart in the method: it measures the
+   implementation. */
 int eb_sampler_set_split_event(eb_sampler_t* h, void* event);
+
+/* Diagnostic hook: the limit, in nanoseconds, of every wait of the stream
+   kernel's pipeline (a consumer waiting for a copy, a producer waiting for a
+   free stage, the hand-off of row records); 0 restores the default of 2 s.
+   A wait that runs out sets EB_STATUS_TIMEOUT, ends the step's stream pass
+   early (the step's outputs are then not valid) and leaves the device
+   usable; the wait for copies still in flight when the kernel exits keeps
+   its own 2 s limit.  Tests use a tiny limit to drive that error path
+   without a fault.  After a timeout, start the canvases again with
+   eb_sampler_init_canvas (which also clears the row counters a cut-short
+   step may leave).  No counterpart in the method. */
+int eb_sampler_set_wait_limit(eb_sampler_t* h, uint64_t limit_ns);
 
 /* Bytes of device workspace the handle holds. */
 size_t eb_sampler_workspace_bytes(const eb_sampler_t* h);

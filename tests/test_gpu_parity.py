@@ -67,10 +67,12 @@ def make_sampler(E, w, **over):
     return E.EBSampler(w.B, w.L, w.V, device=DEV, **cfg)
 
 
-def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=0, mask=None):
+def run_full(E, w, byte_offset=0, canvas_offset=0, max_resyncs=0, mask=None, eb=None):
     """Whole trajectory, every canvas, every position compared with the oracle.
-    `mask(logits, s)` may edit the generated logits in place (e.g. -inf)."""
-    eb = make_sampler(E, w, canvas_offset=canvas_offset)
+    `mask(logits, s)` may edit the generated logits in place (e.g. -inf).
+    `eb`: an existing handle to continue with (it is restarted here)."""
+    if eb is None:
+        eb = make_sampler(E, w, canvas_offset=canvas_offset)
     canvas, committed, stop = eb.new_canvas()
     H, amax = eb.outputs()
     st = O.State(oracle_config(w, canvas_offset=canvas_offset)).init()
@@ -603,3 +605,55 @@ def test_deterministic_and_graph_capture(E):
         for x, y in zip((c, m, st, h, a), r1):
             assert torch.equal(x, y)
     del g
+
+
+# ----------------------------------------------------------------------------- failure paths
+
+def test_timed_out_wait_reports_status_and_the_next_trajectory_matches(E):
+    """A stream-kernel pipeline wait that runs out (limit shortened to 1 ns
+    through the diagnostic hook) sets STATUS_TIMEOUT and returns instead of
+    hanging; after the normal limit is restored and the canvases are started
+    again, a trajectory matches the oracle."""
+    w = MID.replace(B=1, L=16, V=262144, num_steps=3, seed=61)
+    eb = make_sampler(E, w)
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    logits = alloc_logits(w)
+    synth.generate_device(w, 0, logits)
+    eb.set_wait_limit(1)
+    eb.step(logits, 0, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    st = eb.status(clear=True)
+    assert st & E.STATUS_TIMEOUT, st
+    assert eb.status() == 0
+    eb.set_wait_limit(0)
+    stats = run_full(E, w, eb=eb)  # the same handle, started again
+    print(stats)
+
+
+def test_handles_with_different_batch_sizes_coexist(E):
+    """A handle for many canvases keeps working after a handle for one canvas
+    is created on the same device (kernel attributes are per device and are
+    never lowered)."""
+    wb = MID.replace(B=128, L=8, V=300, num_steps=3, seed=62)
+    big = make_sampler(E, wb)
+    small = make_sampler(E, wb.replace(B=1))
+    small.close()
+    canvas, committed, stop = big.new_canvas()
+    H, amax = big.outputs()
+    st = O.State(oracle_config(wb)).init()
+    logits = alloc_logits(wb)
+    for s in range(wb.num_steps):
+        synth.generate_device(wb, s, logits)
+        big.step(logits, s, canvas, committed, H, amax, stop)
+        torch.cuda.synchronize()
+        lg = host_logits(logits)
+        Hg, cvg = H.cpu().numpy(), canvas.cpu().numpy()
+        for i in range(wb.B):
+            out = O.step_canvas(st, i, lg[i], s)
+            if out is None:
+                continue
+            assert np.abs(Hg[i] - out["H"]).max() <= h_tol(False)
+            assert np.array_equal(cvg[i], st.canvas[i])
+    assert big.status() == 0
+    big.close()
