@@ -51,11 +51,22 @@ struct Acc {
   int gb;        // group of R (kNone: none)
 };
 
-// A stream CTA's record of one row: its Acc (32 bytes).
+// A stream CTA's record of one row, final for its part of the row: sums
+// relative to its maximum M, the exact form of its top group (elements equal
+// to M counted, the smaller ones summed), its best Gumbel group and the
+// element drawn inside that group.  48 bytes.
 struct Rec {
-  Acc a;
+  float M;
+  float Sr, Wr;  // every group but the top group
+  float tS, tW;  // the top group's elements below M
+  float R;       // best Gumbel ratio relative to M (0: none)
+  int tn;        // elements of the top group equal to M
+  int ta;        // lowest local id holding M (kNone: no finite logit)
+  int gb;        // group of R (kNone: none)
+  int xs;        // element drawn in group gb (local id; kNone: none)
+  int pad0, pad1;
 };
-static_assert(sizeof(Rec) == 32, "row record layout");
+static_assert(sizeof(Rec) == 48, "row record layout");
 
 // What one vocabulary slice contributes to a position (vocabulary-sharded
 // logits): sums relative to the slice maximum (d = (z - zmax) c2, log2
@@ -87,6 +98,9 @@ struct StepArgs {
   uint32_t* status;
   int32_t* act_index;  // [B] written by the stream kernel: active index or -1
   int32_t* n_act;      // [1] written by the stream kernel
+  int32_t* canvas_cnt;  // [B]: positions of the canvas finished (zero between steps)
+  int32_t* sync_cnt;    // [2]: stream CTAs started, exited (zero between steps)
+  int run_epilogue;     // the stream kernel runs each finished canvas's decisions
   uint64_t wait_ns;    // limit of the stream kernel's pipeline waits
   int B, L, V, ng, s, N;
   int max_segs;  // stream CTAs that can share one row
@@ -254,7 +268,7 @@ __device__ __forceinline__ uint32_t bf16x2_max(uint32_t a, uint32_t b) {
 // 8 ((k + rot) & 7) + 2 i (low half) and + 1 (high half).
 // ---------------------------------------------------------------------------
 #ifndef EB_POLY_PER8
-#define EB_POLY_PER8 2  // words of every 8 whose exponentials use ex2_poly2
+#define EB_POLY_PER8 0  // words of every 8 whose exponentials use ex2_poly2
 #endif
 constexpr int kPolyPer8 = EB_POLY_PER8;
 
@@ -431,13 +445,16 @@ __device__ __forceinline__ float lane_new_top(Acc& A, float mg, int j, float S, 
 // word x).  Since E = -ln u >= 1 - u, a group with Z <= R (1 - u) cannot beat
 // R (checked with a 1e-4 relative margin): its logarithm is skipped.  Strict
 // comparison: on equal ratios the earlier (lower) group stays.
-__device__ __forceinline__ void lane_race(Acc& A, float Z, uint32_t x, int j) {
-  if (Z * 1.0001f <= A.R * one_minus_u(x)) return;
+// Returns true when group j becomes the lane's best.
+__device__ __forceinline__ bool lane_race(Acc& A, float Z, uint32_t x, int j) {
+  if (Z * 1.0001f <= A.R * one_minus_u(x)) return false;
   const float E = -logf(uniform_open(x));
   if (Z > A.R * E) {
     A.R = __fdividef(Z, E);
     A.gb = j;
+    return true;
   }
+  return false;
 }
 
 }  // namespace ebk

@@ -164,6 +164,14 @@ __device__ __forceinline__ int ld_acquire_shared(const int* p) {
   return v;
 }
 
+// Global counter read with acquire semantics at GPU scope (pairs with a
+// writer's fence before its atomic update).
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // Waits (bounded like mbar_wait) until *p > k.
 __device__ __forceinline__ bool wait_counter_above(const int* p, int k,
                                                    uint64_t limit_ns = kWaitLimitNs) {
@@ -231,6 +239,15 @@ __device__ __forceinline__ void griddep_launch_dependents() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Block barrier entered by converged warps.  The barrier instruction counts
+// arrivals per warp-wide instruction, so a warp whose lanes reached it apart
+// (after divergent code) would be counted more than once and could let it
+// complete early; the warp barrier first reconverges the lanes.
+__device__ __forceinline__ void block_sync() {
+  __syncwarp();
+  __syncthreads();
+}
 
 // Named barrier among the consumer warps only (the producer warp never joins).
 __device__ __forceinline__ void consumer_sync(int nthreads) {

@@ -1,12 +1,14 @@
-// eb_finish.cuh -- the per-canvas decisions of a sampler step (the epilogue
-// kernel), the combine of vocabulary-slice records, and the initial canvas.
+// eb_finish.cuh -- the per-canvas decisions of a sampler step (the canvas
+// epilogue), the combine of vocabulary-slice records, and the initial canvas.
 //
-// The stream kernel leaves every position's entropy, argmax, max probability
-// and draw in global memory.  One CTA per canvas then runs the decisions:
-// argmax stability, adaptive stop, commit rule, last-step / all-committed
-// finalisation and renoise.  The entropy-bound rule sorts the candidates by
-// (entropy, position) with a bitonic sort in shared memory and commits the
-// prefix whose float64 running sum stays within the bound.
+// Every position's entropy, argmax, max probability and draw are in global
+// memory when a canvas's decisions run: argmax stability, adaptive stop,
+// commit rule, last-step / all-committed finalisation and renoise.  The
+// stream kernel runs them in the CTA that finishes the canvas's last
+// position; the combine kernel runs them for vocabulary-sharded logits.  The
+// entropy-bound rule sorts the candidates by (entropy, position) with a
+// bitonic sort in shared memory and commits the prefix whose float64 running
+// sum stays within the bound.
 //
 // Pages (cited by title and section): DiffusionGemma model card, "Best
 // practices, 1. Diffusion sampling settings" (lowest-entropy selection under
@@ -22,16 +24,16 @@
 
 namespace ebk {
 
-constexpr int kEpiThreads = 256;
-constexpr int kEpiWarps = kEpiThreads / 32;
+constexpr int kEpiThreads = 256;  // the combine kernel's block
 
+// Scratch of the block-wide helpers (up to 32 warps).
 struct EpiCtrl {
   int stable_prev;
   int pad;
-  double dscr[kEpiWarps];
-  int iscr[kEpiWarps];
-  int cscr[kEpiWarps];
-  unsigned long long uscr[kEpiWarps];
+  double dscr[32];
+  int iscr[32];
+  int cscr[32];
+  unsigned long long uscr[32];
 };
 
 __host__ __device__ inline int pow2_at_least(int n) {
@@ -106,20 +108,22 @@ __device__ __forceinline__ EpiSmem epi_smem(unsigned char* smem, int L) {
 }
 
 // ---------------------------------------------------------------------------
-// Block helpers (kEpiThreads threads, __syncthreads)
+// Block helpers (NT threads, __syncthreads)
 // ---------------------------------------------------------------------------
+template <int NT>
 __device__ __forceinline__ int epi_block_sum_int(int v, EpiCtrl* c) {
   const int tid = threadIdx.x;
 #pragma unroll
   for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   if ((tid & 31) == 0) c->iscr[tid >> 5] = v;
-  __syncthreads();
+  block_sync();
   int r = 0;
-  for (int w = 0; w < kEpiWarps; ++w) r += c->iscr[w];
-  __syncthreads();
+  for (int w = 0; w < NT / 32; ++w) r += c->iscr[w];
+  block_sync();
   return r;
 }
 
+template <int NT>
 __device__ __forceinline__ unsigned long long epi_block_min(unsigned long long v, EpiCtrl* c) {
   const int tid = threadIdx.x;
 #pragma unroll
@@ -128,15 +132,16 @@ __device__ __forceinline__ unsigned long long epi_block_min(unsigned long long v
     v = w < v ? w : v;
   }
   if ((tid & 31) == 0) c->uscr[tid >> 5] = v;
-  __syncthreads();
+  block_sync();
   unsigned long long r = c->uscr[0];
-  for (int w = 1; w < kEpiWarps; ++w) r = c->uscr[w] < r ? c->uscr[w] : r;
-  __syncthreads();
+  for (int w = 1; w < NT / 32; ++w) r = c->uscr[w] < r ? c->uscr[w] : r;
+  block_sync();
   return r;
 }
 
 // One block-wide pass: sum of a (double), OR of b, exclusive prefix of c
 // (*c_total gets the sum of c).
+template <int NT>
 __device__ __forceinline__ void epi_block_reduce(double& a, int& b, int& c, int* c_total,
                                                  EpiCtrl* ctrl) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -157,17 +162,17 @@ __device__ __forceinline__ void epi_block_reduce(double& a, int& b, int& c, int*
     ctrl->iscr[warp] = y;
     ctrl->cscr[warp] = z;
   }
-  __syncthreads();
+  block_sync();
   double sx = 0.0;
   int sy = 0, off = 0, tot = 0;
 #pragma unroll
-  for (int w = 0; w < kEpiWarps; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     sx += ctrl->dscr[w];
     sy |= ctrl->iscr[w];
     if (w < warp) off += ctrl->cscr[w];
     tot += ctrl->cscr[w];
   }
-  __syncthreads();
+  block_sync();
   a = sx;
   b = sy;
   c = off + z - c;
@@ -175,11 +180,12 @@ __device__ __forceinline__ void epi_block_reduce(double& a, int& b, int& c, int*
 }
 
 // Ascending bitonic sort of keys[0, P) (P a power of two).
+template <int NT>
 __device__ __forceinline__ void epi_bitonic_sort(unsigned long long* keys, int P) {
   const int tid = threadIdx.x;
   for (int k = 2; k <= P; k <<= 1) {
     for (int j = k >> 1; j > 0; j >>= 1) {
-      for (int i = tid; i < P; i += kEpiThreads) {
+      for (int i = tid; i < P; i += NT) {
         const int p = i ^ j;
         if (p > i) {
           const unsigned long long x = keys[i], y = keys[p];
@@ -190,18 +196,18 @@ __device__ __forceinline__ void epi_bitonic_sort(unsigned long long* keys, int P
           }
         }
       }
-      __syncthreads();
+      block_sync();
     }
   }
 }
 
 // Inclusive float64 prefix sums cum[i] = sum_{m <= i} val(keys[m]), i < P,
-// with P / kEpiThreads consecutive elements per thread.
-template <class Val>
+// with P / NT consecutive elements per thread.
+template <int NT, class Val>
 __device__ __forceinline__ void epi_prefix_sum(const unsigned long long* keys, double* cum, int P,
                                                Val val, EpiCtrl* ctrl) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int per = (P + kEpiThreads - 1) / kEpiThreads;
+  const int per = (P + NT - 1) / NT;
   const int i0 = tid * per;
   double run = 0.0;
   for (int e = 0; e < per && i0 + e < P; ++e) {
@@ -215,11 +221,47 @@ __device__ __forceinline__ void epi_prefix_sum(const unsigned long long* keys, d
     if (lane >= o) x += t;
   }
   if (lane == 31) ctrl->dscr[warp] = x;
-  __syncthreads();
+  block_sync();
   double off = x - run;
   for (int w = 0; w < warp; ++w) off += ctrl->dscr[w];
   for (int e = 0; e < per && i0 + e < P; ++e) cum[i0 + e] += off;
-  __syncthreads();
+  block_sync();
+}
+
+// Ascending bitonic sort of 32 K keys held by one warp, K consecutive keys
+// per lane (key index lane K + e); partners within a lane are swapped in
+// registers, partners in other lanes are exchanged with shuffles.
+template <int K>
+__device__ __forceinline__ void warp_bitonic_sort(unsigned long long (&v)[K]) {
+  const int lane = threadIdx.x & 31;
+#pragma unroll
+  for (int k = 2; k <= 32 * K; k <<= 1) {
+#pragma unroll
+    for (int j = k >> 1; j > 0; j >>= 1) {
+      if (j < K) {
+#pragma unroll
+        for (int e = 0; e < K; ++e) {
+          if (e & j) continue;
+          const int i = lane * K + e;
+          const bool up = (i & k) == 0;
+          const unsigned long long x = v[e], y = v[e ^ j];
+          if ((x > y) == up) {
+            v[e] = y;
+            v[e ^ j] = x;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < K; ++e) {
+          const int i = lane * K + e;
+          const bool up = (i & k) == 0;
+          const bool lower = (i & j) == 0;
+          const unsigned long long o = __shfl_xor_sync(0xffffffffu, v[e], j / K);
+          v[e] = (lower == up) ? (o < v[e] ? o : v[e]) : (o > v[e] ? o : v[e]);
+        }
+      }
+    }
+  }
 }
 
 // Sort keys: ascending (H, l) (H >= 0, so its float bits order like the
@@ -236,9 +278,54 @@ __device__ __forceinline__ float key_value(unsigned long long k) {
   return __uint_as_float((uint32_t)(k >> 32));
 }
 
+// The commit selection of n_c <= 32 K candidate keys (keys[0, n_c) in shared
+// memory) by one warp: sort, then EB: pick every candidate whose float64
+// prefix sum of entropies (in sorted order) stays <= gamma; BR: pick the
+// first `quota`.
+template <int K>
+__device__ __forceinline__ void warp_select(const StepArgs& a, const unsigned long long* keys,
+                                            int n_c, bool br, uint8_t* pick) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long v[K];
+#pragma unroll
+  for (int e = 0; e < K; ++e) {
+    const int i = lane * K + e;
+    v[e] = i < n_c ? keys[i] : ~0ull;
+  }
+  warp_bitonic_sort<K>(v);
+  if (br) {
+#pragma unroll
+    for (int e = 0; e < K; ++e) {
+      const int i = lane * K + e;
+      if (i < n_c && i < a.quota) pick[(int)(v[e] & 0xffffffffu)] = 1;
+    }
+    return;
+  }
+  double c[K];
+  double run = 0.0;
+#pragma unroll
+  for (int e = 0; e < K; ++e) {
+    run += v[e] == ~0ull ? 0.0 : (double)key_value(v[e]);
+    c[e] = run;
+  }
+  double x = run;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const double t = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += t;
+  }
+  const double off = x - run;
+#pragma unroll
+  for (int e = 0; e < K; ++e) {
+    const int i = lane * K + e;
+    if (i < n_c && off + c[e] <= a.gamma) pick[(int)(v[e] & 0xffffffffu)] = 1;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // Canvas epilogue (one CTA, values of every position in shared memory)
 // ---------------------------------------------------------------------------
+template <int NT>
 __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
   const int tid = threadIdx.x;
   const int L = a.L;
@@ -252,7 +339,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
   double sumH = 0.0;
   int neq = a.s < 1 ? 1 : 0;
   int ncand = 0;
-  for (int l = tid; l < L; l += kEpiThreads) {
+  for (int l = tid; l < L; l += NT) {
     m.pick[l] = 0;
     sumH += (double)m.H[l];
     if (a.s >= 1 && m.am[l] != m.prev[l]) neq = 1;
@@ -267,7 +354,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
   }
   int n_c = 0;
   int pos = ncand;
-  epi_block_reduce(sumH, neq, pos, &n_c, ctrl);
+  epi_block_reduce<NT>(sumH, neq, pos, &n_c, ctrl);
   const int stable_new = neq ? 0 : ctrl->stable_prev + 1;
   const double meanH = sumH / (double)L;
   const bool fired = a.stop_enabled && stable_new >= a.stability_steps && meanH < a.tau;
@@ -275,7 +362,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
 
   if (!fired) {
     const int P = pow2_at_least(n_c > 0 ? n_c : 1);
-    for (int l = tid; l < L; l += kEpiThreads) {
+    for (int l = tid; l < L; l += NT) {
       if (!m.open[l]) continue;
       if (!br) {
         if ((double)m.H[l] <= a.gamma) m.keys[pos++] = key_asc(m.H[l], l);
@@ -285,37 +372,53 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
         m.keys[pos++] = key_desc(m.pm[l], l);
       }
     }
-    for (int i = n_c + tid; i < P; i += kEpiThreads) m.keys[i] = ~0ull;
-    __syncthreads();
-    if (n_c > 1) epi_bitonic_sort(m.keys, P);
-    if (!br) {
-      // EB: the longest prefix in (H, l) order whose entropy sum stays
-      // within gamma (the sums grow along the order)
-      epi_prefix_sum(m.keys, m.cum, P,
-                     [](unsigned long long k) { return k == ~0ull ? 0.0 : (double)key_value(k); },
-                     ctrl);
-      for (int i = tid; i < n_c; i += kEpiThreads)
-        if (m.cum[i] <= a.gamma) m.pick[(int)(m.keys[i] & 0xffffffffu)] = 1;
+    block_sync();
+    if (P <= 256) {
+      // one warp sorts and selects in registers
+      if (tid < 32) {
+        if (P <= 32) {
+          warp_select<1>(a, m.keys, n_c, br, m.pick);
+        } else if (P <= 64) {
+          warp_select<2>(a, m.keys, n_c, br, m.pick);
+        } else if (P <= 128) {
+          warp_select<4>(a, m.keys, n_c, br, m.pick);
+        } else {
+          warp_select<8>(a, m.keys, n_c, br, m.pick);
+        }
+      }
     } else {
-      // BR: the quota goes to the first candidates in (-pmax, l) order
-      for (int i = tid; i < n_c && i < a.quota; i += kEpiThreads)
-        m.pick[(int)(m.keys[i] & 0xffffffffu)] = 1;
+      for (int i = n_c + tid; i < P; i += NT) m.keys[i] = ~0ull;
+      block_sync();
+      epi_bitonic_sort<NT>(m.keys, P);
+      if (!br) {
+        // EB: the longest prefix in (H, l) order whose entropy sum stays
+        // within gamma (the sums grow along the order)
+        epi_prefix_sum<NT>(
+            m.keys, m.cum, P,
+            [](unsigned long long k) { return k == ~0ull ? 0.0 : (double)key_value(k); }, ctrl);
+        for (int i = tid; i < n_c; i += NT)
+          if (m.cum[i] <= a.gamma) m.pick[(int)(m.keys[i] & 0xffffffffu)] = 1;
+      } else {
+        // BR: the quota goes to the first candidates in (-pmax, l) order
+        for (int i = tid; i < n_c && i < a.quota; i += NT)
+          m.pick[(int)(m.keys[i] & 0xffffffffu)] = 1;
+      }
     }
-    __syncthreads();
+    block_sync();
     // EB with no candidate: the single lowest (H, l).  MI: the prefix plus
     // the next open position in (H, l) order.  Candidates (H <= gamma) come
     // before every other open position, so both are the lowest open
     // position left out of the prefix.
     if (!br && (a.rule == kRuleMI || n_c == 0)) {
       unsigned long long best = ~0ull;
-      for (int l = tid; l < L; l += kEpiThreads) {
+      for (int l = tid; l < L; l += NT) {
         if (!m.open[l] || m.pick[l]) continue;
         const unsigned long long kk = key_asc(m.H[l], l);
         best = kk < best ? kk : best;
       }
-      best = epi_block_min(best, ctrl);
+      best = epi_block_min<NT>(best, ctrl);
       if (tid == 0 && best != ~0ull) m.pick[(int)(best & 0xffffffffu)] = 1;
-      __syncthreads();
+      block_sync();
     }
   }
 
@@ -323,7 +426,7 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
   const uint32_t bg = (uint32_t)(a.canvas_offset + bi);
   int left = 0;
   const bool edit = !fired && a.eps_edit >= 0.0;
-  for (int l = tid; l < L; l += kEpiThreads) {
+  for (int l = tid; l < L; l += NT) {
     if (!m.open[l]) {
       // block refinement editing: a committed position whose argmax moved
       // takes it when the argmax is confident enough
@@ -345,18 +448,18 @@ __device__ void canvas_epilogue(const StepArgs& a, int bi, const EpiSmem& m) {
     }
     a.prev_amax[row0 + l] = m.am[l];
   }
-  const int left_tot = epi_block_sum_int(left, ctrl);
+  const int left_tot = epi_block_sum_int<NT>(left, ctrl);
   if (tid == 0) {
     a.stable[bi] = stable_new;
     a.stop_flags[bi] = (uint8_t)(fired ? 1 : last_step ? 3 : left_tot == 0 ? 2 : 0);
   }
 }
 
-// What the previous step left: argmax, tokens, open flags, stability.  The
-// stream kernel of the current step never writes these.
+// What the previous step left: argmax, tokens, open flags, stability.
+template <int NT>
 __device__ __forceinline__ void epi_load_state(const StepArgs& a, int bi, const EpiSmem& m) {
   const size_t row0 = (size_t)bi * (size_t)a.L;
-  for (int l = threadIdx.x; l < a.L; l += kEpiThreads) {
+  for (int l = threadIdx.x; l < a.L; l += NT) {
     m.prev[l] = a.prev_amax[row0 + l];
     m.tok[l] = a.canvas[row0 + l];
     m.open[l] = a.committed[row0 + l] == 0;
@@ -364,25 +467,17 @@ __device__ __forceinline__ void epi_load_state(const StepArgs& a, int bi, const 
   if (threadIdx.x == 0) m.ctrl->stable_prev = a.stable[bi];
 }
 
-// act_index[b]: index of canvas b among the canvases active at the start of
-// the step (-1 if it had stopped), written by the stream kernel.
-__global__ void __launch_bounds__(kEpiThreads) epilogue_kernel(const StepArgs a,
-                                                               const int32_t* act_index) {
-  extern __shared__ __align__(128) unsigned char smem[];
-  const int bi = blockIdx.x;
-  const EpiSmem m = epi_smem(smem, a.L);
-  epi_load_state(a, bi, m);
-  griddep_wait();  // the stream kernel has completed and its writes are visible
-  if (act_index[bi] < 0) return;  // a stopped canvas is untouched
+// This step's per-position results of canvas bi, written by other CTAs
+// (read through L2).
+template <int NT>
+__device__ __forceinline__ void epi_load_rows(const StepArgs& a, int bi, const EpiSmem& m) {
   const size_t row0 = (size_t)bi * (size_t)a.L;
-  for (int l = threadIdx.x; l < a.L; l += kEpiThreads) {
-    m.H[l] = a.H_out[row0 + l];
-    m.am[l] = a.amax_out[row0 + l];
-    m.smp[l] = a.sample[row0 + l];
-    m.pm[l] = a.pmax[row0 + l];
+  for (int l = threadIdx.x; l < a.L; l += NT) {
+    m.H[l] = __ldcg(a.H_out + row0 + l);
+    m.am[l] = __ldcg(a.amax_out + row0 + l);
+    m.smp[l] = __ldcg(a.sample + row0 + l);
+    m.pm[l] = __ldcg(a.pmax + row0 + l);
   }
-  __syncthreads();
-  canvas_epilogue(a, bi, m);
 }
 
 // ---------------------------------------------------------------------------
@@ -400,7 +495,7 @@ __global__ void __launch_bounds__(kEpiThreads) combine_kernel(const StepArgs a,
   const int bi = blockIdx.x;
   if (act_index[bi] < 0) return;  // a stopped canvas is untouched
   const EpiSmem m = epi_smem(smem, a.L);
-  epi_load_state(a, bi, m);
+  epi_load_state<kEpiThreads>(a, bi, m);
   const size_t stride = (size_t)a.B * (size_t)a.L;
   for (int l = threadIdx.x; l < a.L; l += kEpiThreads) {
     const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
@@ -442,15 +537,16 @@ __global__ void __launch_bounds__(kEpiThreads) combine_kernel(const StepArgs a,
     m.smp[l] = smp;
     m.pm[l] = pm;
   }
-  __syncthreads();
-  canvas_epilogue(a, bi, m);
+  block_sync();
+  canvas_epilogue<kEpiThreads>(a, bi, m);
 }
 
 // Initial canvas: uniform-random tokens (stream 2), nothing committed; the
-// stability state and the row counters of the stream kernel start at zero.
+// stability state and the row and canvas counters of the stream kernel
+// start at zero.
 __global__ void init_canvas_kernel(int32_t* canvas, uint8_t* committed, uint8_t* stop_flags,
-                                   int32_t* stable, int32_t* row_cnt, int L, int V,
-                                   int canvas_offset, uint32_t key0, uint32_t key1) {
+                                   int32_t* stable, int32_t* row_cnt, int32_t* canvas_cnt, int L,
+                                   int V, int canvas_offset, uint32_t key0, uint32_t key1) {
   const int bi = blockIdx.x;
   const uint32_t bg = (uint32_t)(canvas_offset + bi);
   for (int l = threadIdx.x; l < L; l += blockDim.x) {
@@ -463,6 +559,7 @@ __global__ void init_canvas_kernel(int32_t* canvas, uint8_t* committed, uint8_t*
   if (threadIdx.x == 0) {
     stop_flags[bi] = 0;
     stable[bi] = 0;
+    canvas_cnt[bi] = 0;
   }
 }
 

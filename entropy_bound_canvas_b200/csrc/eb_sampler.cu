@@ -1,12 +1,12 @@
 // eb_sampler.cu -- host side of the C ABI declared in include/eb_sampler.h.
 //
 // Validation, the device workspace, launch configuration and error codes.
-// A step is two kernels on the caller's stream: the persistent stream kernel
-// (eb_stream.cuh, one CTA per SM: every logit once, and every position's
-// entropy, argmax, max probability and draw) and the epilogue kernel
-// (eb_finish.cuh, one CTA per canvas: the canvas decisions), launched as a
-// programmatic dependent of the first so that its launch overlaps the first
-// one's end.  All the per-step arithmetic runs in those kernels.
+// A step is one kernel on the caller's stream: the persistent stream kernel
+// (eb_stream.cuh, one CTA per SM: every logit once, every position's
+// entropy, argmax, max probability and draw, and each canvas's decisions),
+// launched as a programmatic dependent of the stream's previous kernel so
+// that its set-up overlaps that kernel's end.  All the per-step arithmetic
+// runs in the kernels.
 #include "eb_sampler.h"
 
 #include <cuda_runtime.h>
@@ -64,8 +64,6 @@ void device_setup(DeviceAttrs& d, int device) {
                            cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
       cudaFuncSetAttribute(ebk::stream_kernel<ebk::kBF16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
-      cudaFuncSetAttribute(ebk::epilogue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           optin) != cudaSuccess ||
       cudaFuncSetAttribute(ebk::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin) != cudaSuccess) {
     cudaGetLastError();
@@ -96,7 +94,6 @@ struct eb_sampler {
   int ng = 0;
   int max_segs = 0;  // stream CTAs that can share one row
   KernelCfg k[2];    // stream kernel [dtype]
-  KernelCfg epi;     // epilogue kernel
   KernelCfg combine;  // combine kernel (vocabulary slices)
   int V_tot = 0;      // global vocabulary size
   int slice_step = -1;
@@ -106,6 +103,8 @@ struct eb_sampler {
   size_t ws_bytes = 0;
   Rec* recs = nullptr;
   int32_t* row_cnt = nullptr;
+  int32_t* canvas_cnt = nullptr;
+  int32_t* sync_cnt = nullptr;
   uint32_t* status = nullptr;
   int32_t* act_index = nullptr;
   int32_t* n_act = nullptr;
@@ -114,7 +113,7 @@ struct eb_sampler {
   int32_t* sample = nullptr;
   float* pmax = nullptr;
   int last_step = -1;
-  cudaEvent_t split_event = nullptr;  // recorded between the two kernels when set
+  cudaEvent_t split_event = nullptr;  // recorded after the step's kernel when set
 };
 
 namespace {
@@ -247,13 +246,10 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
     delete h;
     return rc;
   }
-  h->epi.fn = reinterpret_cast<const void*>(&ebk::epilogue_kernel);
-  h->epi.smem = ebk::epi_layout(cfg->L).total;
-  h->epi.grid = cfg->B;
   h->combine.fn = reinterpret_cast<const void*>(&ebk::combine_kernel);
-  h->combine.smem = h->epi.smem;
+  h->combine.smem = ebk::epi_layout(cfg->L).total;
   h->combine.grid = cfg->B;
-  if (h->epi.smem > d->optin) {
+  if (h->combine.smem > d->optin) {
     delete h;
     return EB_ERR_OVERFLOW;
   }
@@ -268,6 +264,10 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   off = align256(off + sizeof(Rec) * BL * (size_t)h->max_segs);
   const size_t o_cnt = off;
   off = align256(off + sizeof(int32_t) * BL);
+  const size_t o_ccnt = off;
+  off = align256(off + sizeof(int32_t) * (size_t)cfg->B);
+  const size_t o_sync = off;
+  off = align256(off + sizeof(int32_t) * 2);
   const size_t o_status = off;
   off = align256(off + sizeof(uint32_t));
   const size_t o_act = off;
@@ -294,6 +294,8 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device) {
   char* base = static_cast<char*>(h->ws);
   h->recs = reinterpret_cast<Rec*>(base + o_rec);
   h->row_cnt = reinterpret_cast<int32_t*>(base + o_cnt);
+  h->canvas_cnt = reinterpret_cast<int32_t*>(base + o_ccnt);
+  h->sync_cnt = reinterpret_cast<int32_t*>(base + o_sync);
   h->status = reinterpret_cast<uint32_t*>(base + o_status);
   h->act_index = reinterpret_cast<int32_t*>(base + o_act);
   h->n_act = h->act_index + cfg->B;
@@ -312,7 +314,8 @@ int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
   if (!guard.ok) return EB_ERR_CUDA;
   const eb_config_t& c = h->cfg;
   ebk::init_canvas_kernel<<<c.B, 256, 0, (cudaStream_t)stream>>>(
-      canvas, committed, stop_flags, h->stable, h->row_cnt, c.L, h->V_tot, c.canvas_offset,
+      canvas, committed, stop_flags, h->stable, h->row_cnt, h->canvas_cnt, c.L, h->V_tot,
+      c.canvas_offset,
       (uint32_t)(c.seed & 0xffffffffu), (uint32_t)(c.seed >> 32));
   if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
   h->last_step = -1;
@@ -340,6 +343,8 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
   std::memset(&a, 0, sizeof(a));
   a.recs = h->recs;
   a.row_cnt = h->row_cnt;
+  a.canvas_cnt = h->canvas_cnt;
+  a.sync_cnt = h->sync_cnt;
   a.prev_amax = h->prev_amax;
   a.stable = h->stable;
   a.sample = h->sample;
@@ -373,20 +378,6 @@ void fill_args(const eb_sampler* h, StepArgs& a, int step) {
   a.key1 = (uint32_t)(c.seed >> 32);
 }
 
-// The stream kernel over `logits` (this device's rows or vocabulary slice).
-int launch_stream(const KernelCfg& kc, StepArgs& a, const void* logits, int dtype, size_t V,
-                  cudaStream_t st) {
-  const size_t elt = dtype == EB_F32 ? 4 : 2;
-  a.logits = logits;
-  a.vec_ok = ((uintptr_t)logits % 16 == 0) && ((V * elt) % 16 == 0) ? 1 : 0;
-  a.G1 = kc.grid;
-  void* args[] = {&a};
-  if (cudaLaunchKernel(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), args, kc.smem, st) !=
-      cudaSuccess)
-    return EB_ERR_CUDA;
-  return EB_OK;
-}
-
 // A kernel launched as a programmatic dependent of the previous one on `st`.
 int launch_dependent(const void* fn, dim3 grid, dim3 block, size_t smem, void** args,
                      cudaStream_t st) {
@@ -402,6 +393,19 @@ int launch_dependent(const void* fn, dim3 grid, dim3 block, size_t smem, void** 
   lc.attrs = attr;
   lc.numAttrs = 1;
   return cudaLaunchKernelExC(&lc, fn, args) == cudaSuccess ? EB_OK : EB_ERR_CUDA;
+}
+
+// The stream kernel over `logits` (this device's rows or vocabulary slice),
+// a programmatic dependent of the stream's previous kernel.
+int launch_stream(const KernelCfg& kc, StepArgs& a, const void* logits, int dtype, size_t V,
+                  cudaStream_t st) {
+  const size_t elt = dtype == EB_F32 ? 4 : 2;
+  a.logits = logits;
+  a.vec_ok = ((uintptr_t)logits % 16 == 0) && ((V * elt) % 16 == 0) ? 1 : 0;
+  a.G1 = kc.grid;
+  void* args[] = {&a};
+  return launch_dependent(kc.fn, dim3(kc.grid), dim3(ebk::stream_threads(dtype)), kc.smem, args,
+                          st);
 }
 
 bool is_slice(const eb_sampler* h) {
@@ -434,16 +438,10 @@ int eb_sampler_step(eb_sampler_t* h, const void* logits, int dtype, int step, in
   a.H_out = entropies;
   a.amax_out = argmax;
   a.stop_flags = stop_flags;
-  int rc = launch_stream(h->k[dtype], a, logits, dtype, (size_t)c.V, st);
+  a.run_epilogue = 1;
+  const int rc = launch_stream(h->k[dtype], a, logits, dtype, (size_t)c.V, st);
   if (rc != EB_OK) return rc;
-
   if (h->split_event && cudaEventRecord(h->split_event, st) != cudaSuccess) return EB_ERR_CUDA;
-
-  const int32_t* act_index = h->act_index;
-  void* eargs[] = {&a, &act_index};
-  rc = launch_dependent(h->epi.fn, dim3(h->epi.grid), dim3(ebk::kEpiThreads), h->epi.smem, eargs,
-                        st);
-  if (rc != EB_OK) return rc;
   h->last_step = step;
   return EB_OK;
 }

@@ -21,15 +21,21 @@
 //     When a warp leaves a row it merges its lanes and deposits one record
 //     per row of the CTA's range into a shared-memory slot;
 //   - the finisher warp merges the twelve deposits of each row into the
-//     CTA's record.  A row spread over several CTAs exchanges records through
-//     global memory: each CTA writes its record and counts itself in the
-//     row's counter; the last one merges them all (in CTA order) and
-//     finishes the row: entropy, max probability, argmax, and for an open
-//     position the element draw inside the winning Gumbel group.
-// The per-canvas decisions run in the epilogue kernel (eb_finish.cuh).
+//     CTA's part of the row, made final (the exact top group and the element
+//     drawn in its best Gumbel group).  A row spread over several CTAs
+//     exchanges these records through global memory: each CTA writes its
+//     record and counts itself in the row's counter (or sees that the others
+//     are done already); the last one combines them (in CTA order) and
+//     writes the position's entropy, max probability, argmax and draw.
+// The CTA that finishes a canvas's last position then runs that canvas's
+// decisions with all its threads (eb_finish.cuh), once every CTA of the
+// grid has read the stop flags.  Consecutive steps' kernels are chained by
+// programmatic dependent launch: a CTA sets up its shared memory while the
+// previous step's kernel drains, then waits for it (griddepcontrol.wait).
 #pragma once
 
 #include "eb_common.cuh"
+#include "eb_finish.cuh"
 
 namespace ebk {
 
@@ -37,10 +43,13 @@ namespace ebk {
 #define EB_STREAM_CONSUMER_WARPS 12
 #endif
 #ifndef EB_STREAM_STAGES
-#define EB_STREAM_STAGES 6
+#define EB_STREAM_STAGES 3
 #endif
 #ifndef EB_STREAM_STAGE_KB
-#define EB_STREAM_STAGE_KB 32
+#define EB_STREAM_STAGE_KB 64
+#endif
+#ifndef EB_STREAM_FINISHERS
+#define EB_STREAM_FINISHERS 2
 #endif
 
 constexpr int kStages = EB_STREAM_STAGES;
@@ -49,8 +58,9 @@ constexpr int kSlots = 8;  // row slots of the consumer -> finisher hand-off
 template <int DT>
 struct StreamShape {
   static constexpr int kConsumerWarps = EB_STREAM_CONSUMER_WARPS;
-  // + copy producer, word producer, finisher
-  static constexpr int kThreads = (kConsumerWarps + 3) * 32;
+  static constexpr int kFinishers = EB_STREAM_FINISHERS;  // finisher warps, alternating rows
+  // + copy producer, word producer, finishers
+  static constexpr int kThreads = (kConsumerWarps + 2 + kFinishers) * 32;
   static constexpr int kStageBytes = EB_STREAM_STAGE_KB * 1024;
   // room for a copy widened to 16-byte boundaries; 128-byte aligned stages
   static constexpr int kStageStride = kStageBytes + 128;
@@ -71,6 +81,8 @@ struct StreamCtrl {
   int issued;  // tiles whose bulk copy has been issued
   int n_sub;   // sub-tiles of this CTA's range
   int words_arrived;  // tiles whose second (header) arrival was made
+  int n_epi;          // canvases whose decisions this CTA runs
+  int epi_ok;         // every CTA of the grid has read the stop flags
   int wcnt[32];
 };
 
@@ -95,7 +107,7 @@ struct RowSlot {
 };
 
 struct StreamLayout {
-  uint32_t bars, ctrl, meta, words, slots, act, ring, total;
+  uint32_t bars, ctrl, meta, words, slots, act, epi, ring, total;
 };
 
 __host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
@@ -116,6 +128,8 @@ __host__ __device__ inline StreamLayout stream_layout(int B) {
   y.slots = o;
   o = align_up(o + (uint32_t)sizeof(RowSlot) * kSlots, 16);
   y.act = o;
+  o = align_up(o + 2u * (uint32_t)B, 16);
+  y.epi = o;
   o = align_up(o + 2u * (uint32_t)B, 128);
   y.ring = o;
   o += (uint32_t)kStages * (uint32_t)Sh::kStageStride;
@@ -200,12 +214,12 @@ __device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int 
     const bool on = b < B && __ldcg(stop_flags + b) == 0;
     const unsigned bal = __ballot_sync(0xffffffffu, on);
     if (lane == 0) wcnt[warp] = __popc(bal);
-    __syncthreads();
+    block_sync();
     int off = base;
     for (int w = 0; w < warp; ++w) off += wcnt[w];
     if (on) act[off + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)b;
     for (int w = 0; w < nwarps; ++w) base += wcnt[w];
-    __syncthreads();
+    block_sync();
   }
   return base;
 }
@@ -234,85 +248,10 @@ __device__ __forceinline__ RowSpan row_span(unsigned long long r, int ng, unsign
 }
 
 // ---------------------------------------------------------------------------
-// Finishing a row (one warp): the merged state of all its groups -> the
-// position's outputs.  Entropy and max probability in float64 from the
-// exact top-group count and the small sums; the element draw inside the
-// winning group reads that group's 64 logits and their element-stream
-// Philox words: the largest tempered logit is drawn first, and the
-// logarithms of every element that provably cannot beat it are skipped.
+// A stream CTA's part of a row, made final (one warp): the exact form of its
+// top group and the element draw inside its best Gumbel group, from those
+// two groups' logits (global memory) and their element-stream Philox words.
 // ---------------------------------------------------------------------------
-// The final combine of a row's n records, in stream-CTA order (which is
-// group order): the row maximum, the record holding its top group (the
-// first record attaining it), every record's sums rescaled to the maximum
-// in float64 -- except the top record's top-group sums, which the exact
-// recomputation replaces -- and the best Gumbel ratio (lower group on equal
-// ratios).  `rec(i)` loads record i; every lane returns the same values.
-struct RowFinal {
-  double S, W;  // relative to M, W in log2 units, without the top group
-  float M;
-  int tj;       // top group (local id; kNone: no finite logit)
-  float R;      // best ratio relative to M
-  int gb;       // its group (kNone: none)
-};
-
-template <class Load>
-__device__ __forceinline__ RowFinal combine_records(int n, Load rec, float c2) {
-  float M = -INFINITY;
-  for (int i = threadIdx.x & 31; i < n; i += 32) M = fmaxf(M, rec(i).M);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  // the top record: the first whose maximum is M
-  int top = kNone;
-  for (int i = threadIdx.x & 31; i < n; i += 32)
-    if (rec(i).M == M && M > -INFINITY) top = min(top, i);
-#pragma unroll
-  for (int o = 16; o; o >>= 1) top = min(top, __shfl_xor_sync(0xffffffffu, top, o));
-  double S = 0.0, W = 0.0;
-  float Rl = 0.f;
-  int gl = kNone, tj = kNone;
-  for (int i = threadIdx.x & 31; i < n; i += 32) {
-    const Acc c = rec(i);
-    if (!(c.M > -INFINITY)) continue;
-    const bool tie = c.M == M;
-    const double dd = tie ? 0.0 : (double)((c.M - M) * c2);
-    const double f = tie ? 1.0 : exp2(dd);
-    double So = (double)c.Sr, Wo = (double)c.Wr;
-    if (i == top) {
-      tj = c.tj;
-    } else {
-      So += (double)c.tS;
-      Wo += (double)c.tW;
-    }
-    S += f * So;
-    W += f * (Wo + dd * So);
-    const float Rc = c.R * (float)f;
-    if (Rc > Rl || (Rc == Rl && Rc > 0.f && c.gb < gl)) {
-      Rl = Rc;
-      gl = c.gb;
-    }
-  }
-#pragma unroll
-  for (int o = 16; o; o >>= 1) {
-    S += __shfl_xor_sync(0xffffffffu, S, o);
-    W += __shfl_xor_sync(0xffffffffu, W, o);
-    const float oR = __shfl_xor_sync(0xffffffffu, Rl, o);
-    const int og = __shfl_xor_sync(0xffffffffu, gl, o);
-    if (oR > Rl || (oR == Rl && oR > 0.f && og < gl)) {
-      Rl = oR;
-      gl = og;
-    }
-    tj = min(tj, __shfl_xor_sync(0xffffffffu, tj, o));
-  }
-  RowFinal f;
-  f.S = S;
-  f.W = W;
-  f.M = M;
-  f.tj = tj;
-  f.R = Rl;
-  f.gb = gl;
-  return f;
-}
-
 // This lane's two elements 2 lane, 2 lane + 1 of group j of a row (local
 // ids; those at or beyond V read as -inf).
 template <int DT>
@@ -405,28 +344,36 @@ __device__ __forceinline__ int draw_in_group(const StepArgs& a, float2 z, int j,
   return barg;
 }
 
-// Finishes row (bi, l) from the combined records (one warp): the exact form
-// of the top group (elements equal to the row maximum count 1 each, the
-// smaller ones are summed with d = (z - M) c2 from the exact difference)
-// gives, with the other sums, the entropy and max probability in float64
-// and the argmax; an open position draws inside the winning group.  Writes
-// the position's outputs (or, for a vocabulary slice, its slice record).
+// The CTA's merged state of its part of a row -> its final record, in two
+// halves so that other memory traffic can be issued between them: the loads
+// of the part's top group and best Gumbel group, then the arithmetic.  The
+// top group is recomputed exactly relative to M: elements equal to M count 1
+// each (d = (z - M) c2 from the exact difference), the smaller ones are
+// summed, zero terms skipped.  Every lane returns the record.
+struct PartLoads {
+  float2 zt, zd;
+  bool has, drw;
+};
+
 template <int DT>
-__device__ __forceinline__ void finish_position(const StepArgs& a, const RowFinal& F, int bi, int l,
-                                                bool open) {
+__device__ __forceinline__ PartLoads part_loads(const StepArgs& a, const Acc& A, const char* rowp,
+                                                bool draw) {
+  PartLoads p;
+  p.has = A.M > -INFINITY && A.tj != kNone;
+  p.drw = draw && p.has && A.gb != kNone;
+  p.zt = p.zd = make_float2(-INFINITY, -INFINITY);
+  if (p.has) p.zt = load_pair<DT>(a, rowp, A.tj);
+  if (p.drw) p.zd = load_pair<DT>(a, rowp, A.gb);
+  return p;
+}
+
+__device__ __forceinline__ Rec part_finalize(const StepArgs& a, const Acc& A, const PartLoads& p,
+                                             int bi, int l) {
   const int lane = threadIdx.x & 31;
-  const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
-  const char* rowp =
-      reinterpret_cast<const char*>(a.logits) + grow * (size_t)a.V * (size_t)elt_bytes(DT);
-  const bool draw = open && !a.greedy && F.gb != kNone;
-  // both groups' loads in flight together
-  float2 zt = make_float2(-INFINITY, -INFINITY), zd = zt;
-  if (F.tj != kNone) zt = load_pair<DT>(a, rowp, F.tj);
-  if (draw) zd = load_pair<DT>(a, rowp, F.gb);
   Exact e{0.f, 0.f, 0, kNone};
-  if (F.tj != kNone) {
-    exact_elem(zt.x, F.tj * kGroup + 2 * lane, F.M, a.c2, e);
-    exact_elem(zt.y, F.tj * kGroup + 2 * lane + 1, F.M, a.c2, e);
+  if (p.has) {
+    exact_elem(p.zt.x, A.tj * kGroup + 2 * lane, A.M, a.c2, e);
+    exact_elem(p.zt.y, A.tj * kGroup + 2 * lane + 1, A.M, a.c2, e);
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) {
@@ -435,15 +382,125 @@ __device__ __forceinline__ void finish_position(const StepArgs& a, const RowFina
     e.n += __shfl_xor_sync(0xffffffffu, e.n, o);
     e.amin = min(e.amin, __shfl_xor_sync(0xffffffffu, e.amin, o));
   }
-  int x = kNone;
-  if (draw) x = draw_in_group(a, zd, F.gb, bi, l);
-  if (lane != 0) return;
-  const double S = (double)e.n + ((double)e.S + F.S);
-  const double W = (double)e.W + F.W;
-  const bool bad = !isfinite(S) || !isfinite(W) || F.tj == kNone || e.amin == kNone;
-  if (bad) atomicOr(a.status, kStatusNonFinite);
-  const int amax = e.amin == kNone ? kNone : e.amin + a.v_off;
-  const int smp = x == kNone ? kNone : x + a.v_off;
+  Rec r;
+  r.M = p.has ? A.M : -INFINITY;
+  r.Sr = A.Sr;
+  r.Wr = A.Wr;
+  r.tS = e.S;
+  r.tW = e.W;
+  r.R = A.R;
+  r.tn = e.n;
+  r.ta = e.amin;
+  r.gb = A.gb;
+  r.xs = p.drw ? draw_in_group(a, p.zd, A.gb, bi, l) : kNone;
+  r.pad0 = r.pad1 = 0;
+  return r;
+}
+
+__device__ __forceinline__ Rec ld_rec(const Rec* p) {
+  Rec r;
+  const float4 u = __ldcg(reinterpret_cast<const float4*>(p));
+  const float4 v = __ldcg(reinterpret_cast<const float4*>(p) + 1);
+  const int4 w = __ldcg(reinterpret_cast<const int4*>(p) + 2);
+  r.M = u.x;
+  r.Sr = u.y;
+  r.Wr = u.z;
+  r.tS = u.w;
+  r.tW = v.x;
+  r.R = v.y;
+  r.tn = __float_as_int(v.z);
+  r.ta = __float_as_int(v.w);
+  r.gb = w.x;
+  r.xs = w.y;
+  r.pad0 = r.pad1 = 0;
+  return r;
+}
+
+// The row's n records in stream-CTA order (which is group order), combined
+// in float64: the row maximum M; the first record attaining it gives the
+// argmax; every record's sums are rescaled to M (a record whose maximum
+// equals M adds its count of maxima exactly); the best Gumbel ratio (lower
+// group on equal ratios) gives the draw.  `rec(i)` returns record i; every
+// lane returns the same values.
+struct RowFinal {
+  double S, W;  // relative to M, W in log2 units
+  float M, R;
+  int amax, gb, xs;  // local ids
+};
+
+template <class Load>
+__device__ __forceinline__ RowFinal combine_records(int n, Load rec, float c2) {
+  const int lane = threadIdx.x & 31;
+  float M = -INFINITY;
+  for (int i = lane; i < n; i += 32) M = fmaxf(M, rec(i).M);
+#pragma unroll
+  for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+  double S = 0.0, W = 0.0;
+  float Rl = 0.f;
+  int gl = kNone, xl = kNone, top = kNone, ta = kNone;
+  for (int i = lane; i < n; i += 32) {
+    const Rec c = rec(i);
+    if (!(c.M > -INFINITY)) continue;
+    const bool tie = c.M == M;
+    if (tie && i < top) {
+      top = i;
+      ta = c.ta;
+    }
+    const double dd = tie ? 0.0 : (double)((c.M - M) * c2);
+    const double f = tie ? 1.0 : exp2(dd);
+    const double So = (double)c.tn + ((double)c.tS + (double)c.Sr);
+    const double Wo = (double)c.tW + (double)c.Wr;
+    S += f * So;
+    W += f * (Wo + dd * So);
+    const float Rc = c.R * (float)f;
+    if (Rc > Rl || (Rc == Rl && Rc > 0.f && c.gb < gl)) {
+      Rl = Rc;
+      gl = c.gb;
+      xl = c.xs;
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) {
+    S += __shfl_xor_sync(0xffffffffu, S, o);
+    W += __shfl_xor_sync(0xffffffffu, W, o);
+    const float oR = __shfl_xor_sync(0xffffffffu, Rl, o);
+    const int og = __shfl_xor_sync(0xffffffffu, gl, o);
+    const int ox = __shfl_xor_sync(0xffffffffu, xl, o);
+    if (oR > Rl || (oR == Rl && oR > 0.f && og < gl)) {
+      Rl = oR;
+      gl = og;
+      xl = ox;
+    }
+    const int ot = __shfl_xor_sync(0xffffffffu, top, o);
+    const int oa = __shfl_xor_sync(0xffffffffu, ta, o);
+    if (ot < top) {
+      top = ot;
+      ta = oa;
+    }
+  }
+  RowFinal f;
+  f.S = S;
+  f.W = W;
+  f.M = M;
+  f.R = Rl;
+  f.amax = ta;
+  f.gb = gl;
+  f.xs = xl;
+  return f;
+}
+
+// The position's outputs from its combined records (lane 0 writes): the
+// entropy and max probability in float64, the argmax, the draw -- or, for a
+// vocabulary slice, its slice record.
+__device__ __forceinline__ void write_position(const StepArgs& a, const RowFinal& F, int bi, int l,
+                                               bool open) {
+  if ((threadIdx.x & 31) != 0) return;
+  const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
+  const double S = F.S, W = F.W;
+  if (!isfinite(S) || !isfinite(W) || F.amax == kNone) atomicOr(a.status, kStatusNonFinite);
+  const int amax = F.amax == kNone ? kNone : F.amax + a.v_off;
+  const bool drawn = open && !a.greedy && F.xs != kNone;
+  const int smp = drawn ? F.xs + a.v_off : amax;
   if (a.slice_out != nullptr) {
     SliceRecord r;
     r.S = S;
@@ -451,7 +508,7 @@ __device__ __forceinline__ void finish_position(const StepArgs& a, const RowFina
     r.zmax = F.M;
     r.gscore = (F.R > 0.f && F.gb != kNone) ? fmaf(F.M, a.iT, logf(F.R)) : -INFINITY;
     r.amax = amax;
-    r.sample = draw ? smp : -1;
+    r.sample = drawn ? smp : -1;
     r.pad0 = r.pad1 = 0;
     a.slice_out[grow] = r;
     return;
@@ -459,7 +516,7 @@ __device__ __forceinline__ void finish_position(const StepArgs& a, const RowFina
   a.H_out[grow] = (float)(log(S) - 0.6931471805599453 * (W / S));
   a.amax_out[grow] = amax;
   a.pmax[grow] = (float)(1.0 / S);
-  a.sample[grow] = open ? (draw ? smp : amax) : -1;
+  a.sample[grow] = open ? smp : -1;
 }
 
 // One CTA per SM: the register cap is the register file over the block.
@@ -476,6 +533,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + lay.words);
   RowSlot* slots = reinterpret_cast<RowSlot*>(smem + lay.slots);
   uint16_t* act = reinterpret_cast<uint16_t*>(smem + lay.act);
+  uint16_t* epi = reinterpret_cast<uint16_t*>(smem + lay.epi);
   unsigned char* ring = smem + lay.ring;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -487,16 +545,23 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     ctrl->abort = 0;
     ctrl->issued = 0;
     ctrl->words_arrived = 0;
+    ctrl->n_epi = 0;
+    ctrl->epi_ok = 0;
     for (int i = 0; i < kSlots; ++i) {
       slots[i].q = i;
       slots[i].count = 0;
     }
     fence_mbar_init();
   }
+  // Everything above is this CTA's own shared memory; from here on the
+  // kernel reads what the previous step's kernel wrote (stop flags, canvas
+  // state, counters): wait until that grid has completed.
+  griddep_wait();
   const int n_act = build_active_list(a.stop_flags, a.B, act, ctrl->wcnt, Sh::kThreads);
+  if (a.run_epilogue && tid == 0) atomicAdd(a.sync_cnt, 1);  // this CTA has read the stop flags
   if (blockIdx.x == 0) {  // publish the active list for the epilogue kernel
     for (int b = tid; b < a.B; b += Sh::kThreads) a.act_index[b] = -1;
-    __syncthreads();
+    block_sync();
     for (int i = tid; i < n_act; i += Sh::kThreads) a.act_index[act[i]] = i;
     if (tid == 0) *a.n_act = n_act;
   }
@@ -506,10 +571,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   const unsigned long long g_lo = range_start(blockIdx.x, NG, G);
   const unsigned long long g_hi = range_start(blockIdx.x + 1, NG, G);
   if (tid == 0) ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
-  __syncthreads();
-  // The epilogue kernel may be scheduled from now on, wherever an SM has
-  // room: its CTAs load what the previous step left and then wait for this
-  // grid's completion (griddepcontrol.wait) before reading anything it writes.
+  block_sync();
+  // The next kernel on the stream may be scheduled from now on, wherever an
+  // SM has room: it waits for this grid's completion (griddepcontrol.wait)
+  // before reading anything this grid writes.
   griddep_launch_dependents();
 
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
@@ -517,19 +582,27 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   const long long r_first = (long long)(g_lo / (unsigned long long)a.ng);
   const long long r_end =
       g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
+  auto row_of = [&](long long r, int& bi, int& l) {
+    const int ai = (int)(r / a.L);
+    l = (int)(r - (long long)ai * a.L);
+    bi = act[ai];
+  };
 
   if (warp == NW) {
     // ------------------------------------------------------- copy producer
     // Lane 0 alone: waits for a free stage, issues the tile's bulk copy (the
-    // stage's first arrival, with the bytes) and writes its description.
+    // stage's first arrival, with the bytes) and writes its description.  No
+    // global load ever delays the next copy.
     if (lane == 0) {
+      // Logits are read once: L2 evict-first, so that the stream does not push
+      // out the kernel's code and small state.
       const uint64_t policy = evict_first_policy();
       TileIter it(g_lo, g_hi, a.ng, a.L, Sh::kStageGroups);
       Tile t;
       int k = 0, st = 0;
       uint32_t ph = 0;  // parity of the current pass over the ring
       long long row_seen = -1;
-      int bi = 0, samp = 0;
+      int bi = 0;
       while (it.next(t)) {
         if (k >= kStages && !mbar_wait(&empty[st], ph ^ 1u, a.wait_ns)) {
           atomicOr(a.status, kStatusTimeout);
@@ -537,8 +610,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           break;
         }
         if (*(volatile int*)&ctrl->abort) break;
-        const bool new_row = t.r != row_seen;
-        if (new_row) {
+        if (t.r != row_seen) {
           row_seen = t.r;
           bi = act[t.ai];
         }
@@ -555,16 +627,13 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         mbar_arrive_expect_tx(&full[st], (uint32_t)(a1 - a0));
         bulk_load(ring + (size_t)st * Sh::kStageStride, reinterpret_cast<const void*>(a0),
                   (uint32_t)(a1 - a0), &full[st], policy);
-        // The position's committed flag is read while the copy is in flight.
-        if (new_row)
-          samp = !a.greedy && a.committed[(size_t)bi * (size_t)a.L + (size_t)t.l] == 0;
         TileMeta m;
         m.r = (int)t.r;
         m.j0 = t.j0;
         m.cnt = t.cnt;
         m.bi = bi;
         m.l = t.l;
-        m.sampling = samp;
+        m.sampling = 0;  // set by the word producer
         m.delta = (int)(reinterpret_cast<uintptr_t>(src) - a0);
         m.pad = 0;
         meta[st] = m;
@@ -575,14 +644,33 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           ph ^= 1u;
         }
       }
+      // Have all CTAs of the grid read the stop flags?  (Checked here, long
+      // before this CTA can need it, so that a canvas's decisions at the end
+      // rarely wait for the round trip.)
+      if (a.run_epilogue && ld_acquire_gpu(a.sync_cnt) >= (int)gridDim.x) ctrl->epi_ok = 1;
     }
   } else if (warp == NW + 1) {
     // ------------------------------------------------------- word producer
     // Once tile k is issued (its stage free and its description written),
-    // computes the group-stream Philox words of an open position's groups
-    // into the stage's header and makes the stage's second arrival.
+    // decides whether its position draws (open, not greedy), computes the
+    // group-stream Philox words of a drawing position's groups into the
+    // stage's header and makes the stage's second arrival.  The committed
+    // flags of the range's first 32 rows are loaded at once, at the start.
     const int n_tiles = ctrl->n_sub / Sh::kSubPerStage;
+    uint32_t open_bits = 0;
+    if (!a.greedy) {
+      const long long r = r_first + lane;
+      bool o = false;
+      if (r < r_end) {
+        int bi, l;
+        row_of(r, bi, l);
+        o = a.committed[(size_t)bi * (size_t)a.L + (size_t)l] == 0;
+      }
+      open_bits = __ballot_sync(0xffffffffu, o);
+    }
     int st = 0, words_done = 0;
+    long long row_seen = -1;
+    int samp = 0;
     for (int k = 0; k < n_tiles; ++k, words_done = k) {
       if (!wait_counter_above(&ctrl->issued, k, a.wait_ns)) {
         if (lane == 0) {
@@ -591,37 +679,58 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         }
         break;
       }
-      const TileMeta m = meta[st];
-      if (m.sampling) {
+      TileMeta* mp = &meta[st];
+      const int mr = mp->r, mj0 = mp->j0, mcnt = mp->cnt, mbi = mp->bi, ml = mp->l;
+      if (mr != row_seen) {
+        row_seen = mr;
+        const long long q = mr - r_first;
+        samp = !a.greedy &&
+               (q < 32 ? (open_bits >> q) & 1u
+                       : a.committed[(size_t)mbi * (size_t)a.L + (size_t)ml] == 0);
+      }
+      if (samp) {
         uint32_t* wd = words + st * Sh::kStageGroups;
-        const int gj0 = (a.v_off >> 6) + m.j0;  // global group id of the tile's first group
-        const int c0 = gj0 >> 2, c1 = (gj0 + m.cnt - 1) >> 2;
-        const uint32_t c3 = (uint32_t)(a.canvas_offset + m.bi) | (kStreamGroup << 24);
+        const int gj0 = (a.v_off >> 6) + mj0;  // global group id of the tile's first group
+        const int c0 = gj0 >> 2, c1 = (gj0 + mcnt - 1) >> 2;
+        const uint32_t c3 = (uint32_t)(a.canvas_offset + mbi) | (kStreamGroup << 24);
         for (int c = c0 + lane; c <= c1; c += 32) {
-          const Words4 w = philox((uint32_t)c, (uint32_t)m.l, (uint32_t)a.s, c3, a.key0, a.key1);
+          const Words4 w = philox((uint32_t)c, (uint32_t)ml, (uint32_t)a.s, c3, a.key0, a.key1);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int j = 4 * c + q - gj0;
-            if (j >= 0 && j < m.cnt) wd[j] = w.w[q];
+            if (j >= 0 && j < mcnt) wd[j] = w.w[q];
           }
         }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&full[st]);  // header (words) complete
+      if (lane == 0) {
+        mp->sampling = samp;
+        mbar_arrive(&full[st]);  // header (words, draw flag) complete
+      }
       if (++st == kStages) st = 0;
     }
     if (lane == 0) ctrl->words_arrived = words_done;
-  } else if (warp == NW + 2) {
-    // ------------------------------------------------------------ finisher
+  } else if (warp >= NW + 2) {
+    // ----------------------------------------------------------- finishers
+    // Finisher f takes the rows q = f, f + kFinishers, ... of the range, so
+    // that rows completed close together (at the end of the range) are
+    // finished in parallel.
     const int nrows = (int)(r_end - r_first);
-    for (int q = 0; q < nrows; ++q) {
+    const int f = warp - (NW + 2);
+    for (int q = f; q < nrows; q += Sh::kFinishers) {
       RowSlot* sl = &slots[q % kSlots];
       const long long r = r_first + q;
-      const int ai = (int)(r / a.L);
-      const int l = (int)(r - (long long)ai * a.L);
-      const int bi = act[ai];
+      int bi, l;
+      row_of(r, bi, l);
       const size_t grow = (size_t)bi * (size_t)a.L + (size_t)l;
       const bool open = a.committed != nullptr && a.committed[grow] == 0;
+      const RowSpan sp = row_span((unsigned long long)r, a.ng, NG, G, blockIdx.x);
+      Rec* rr = a.recs + grow * (size_t)a.max_segs;
+      // Are the row's other stream CTAs done already?  (Read before this
+      // CTA's part is ready; if so, this CTA finishes the row without the
+      // counter's round trip.)
+      int pre = 0;
+      if (sp.nseg > 1 && lane == 0) pre = ld_acquire_gpu(a.row_cnt + grow);
       // the twelve deposits of row q
       bool ok = true;
       {
@@ -647,48 +756,62 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       } else {
         acc_reset(mine);
       }
-      warp_merge_acc(mine, a.c2, 16);
+      warp_merge_acc(mine, a.c2);  // every lane ends with the CTA's merged state
       __syncwarp();
       if (lane == 0) {
         sl->count = 0;
         st_release_shared(&sl->q, q + kSlots);
       }
-      // the row's other stream CTAs
-      const RowSpan sp = row_span((unsigned long long)r, a.ng, NG, G, blockIdx.x);
+      const char* rowp = logits + grow * row_bytes;
+      // this part's candidate groups: loads in flight first
+      const PartLoads pl = part_loads<DT>(a, mine, rowp, open && !a.greedy);
+      // then the row's counter again if the early read did not show the other
+      // CTAs done (they usually are by now), and their records
+      if (sp.nseg > 1 && lane == 0 && pre != sp.nseg - 1) pre = ld_acquire_gpu(a.row_cnt + grow);
+      const bool others_done =
+          sp.nseg > 1 && __shfl_sync(0xffffffffu, pre, 0) == sp.nseg - 1;
+      Rec other;
+      other.M = -INFINITY;
+      if (others_done && lane < sp.nseg && lane != sp.seg) other = ld_rec(rr + lane);
+      const Rec own = part_finalize(a, mine, pl, bi, l);
+      // the canvas's finished positions; the CTA finishing its last one runs
+      // the canvas's decisions after its roles are done
+      auto count_canvas = [&]() {
+        if (!a.run_epilogue || lane != 0) return;
+        __threadfence();
+        if (atomicAdd(a.canvas_cnt + bi, 1) == a.L - 1) {
+          __threadfence();
+          epi[atomicAdd(&ctrl->n_epi, 1)] = (uint16_t)bi;
+        }
+      };
       if (sp.nseg == 1) {
-        // lanes below 16 hold the CTA's merged state
-        const RowFinal F = combine_records(1, [&](int) { return mine; }, a.c2);
-        finish_position<DT>(a, F, bi, l, open);
+        const RowFinal F = combine_records(1, [&](int) { return own; }, a.c2);
+        write_position(a, F, bi, l, open);
+        count_canvas();
         continue;
       }
-      Rec* rr = a.recs + grow * (size_t)a.max_segs;
-      int last = 0;
-      if (lane == 0) {
-        Rec w;
-        w.a = mine;
-        rr[sp.seg] = w;
+      bool last = others_done;
+      if (!last) {
+        int old = 0;
+        if (lane == 0) {
+          rr[sp.seg] = own;
+          __threadfence();
+          old = atomicAdd(a.row_cnt + grow, 1);
+        }
+        last = __shfl_sync(0xffffffffu, old, 0) == sp.nseg - 1;
+        if (!last) continue;
         __threadfence();
-        last = atomicAdd(a.row_cnt + grow, 1) == sp.nseg - 1;
+        if (lane < sp.nseg && lane != sp.seg) other = ld_rec(rr + lane);
       }
-      last = __shfl_sync(0xffffffffu, last, 0);
-      if (!last) continue;
-      __threadfence();
-      auto load = [&](int i) {
-        const Acc* p = &rr[i].a;
-        Acc c;
-        c.M = __ldcg(&p->M);
-        c.tS = __ldcg(&p->tS);
-        c.tW = __ldcg(&p->tW);
-        c.Sr = __ldcg(&p->Sr);
-        c.Wr = __ldcg(&p->Wr);
-        c.R = __ldcg(&p->R);
-        c.tj = __ldcg(&p->tj);
-        c.gb = __ldcg(&p->gb);
-        return c;
+      auto rec = [&](int i) -> Rec {
+        if (i == sp.seg) return own;
+        if (i < 32) return other;  // lane i holds record i
+        return ld_rec(rr + i);
       };
-      const RowFinal F = combine_records(sp.nseg, load, a.c2);
+      const RowFinal F = combine_records(sp.nseg, rec, a.c2);
       if (lane == 0) a.row_cnt[grow] = 0;  // zero again for the next step
-      finish_position<DT>(a, F, bi, l, open);
+      write_position(a, F, bi, l, open);
+      count_canvas();
     }
   } else {
     // ------------------------------------------------------------ consumers
@@ -701,8 +824,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     const int rot = lane;
     bool fail = false;
 
-    // This warp's record of CTA-relative row q into its slot (after the
-    // finisher has released the slot's previous row).
+    // This warp's record of row r into its slot (after the finisher has
+    // released the slot's previous row).
     auto deposit = [&](long long r, bool empty_rec) -> bool {
       Acc w = A;
       if (!empty_rec) warp_merge_acc(w, a.c2);
@@ -734,43 +857,38 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         if (!deposit(next_r, true)) return false;
       return true;
     };
+    // A row change: this warp's deposit of the row it leaves, empty ones for
+    // the rows of the range it skipped, and a fresh state.
+    auto enter_row = [&](const TileMeta& m) -> bool {
+      if (m.r == cur_r) return true;
+      if (cur_r >= 0) {
+        if (!deposit(cur_r, false)) return false;
+        next_r = cur_r + 1;
+      }
+      if (!owe_empty(m.r)) return false;
+      cur_r = m.r;
+      next_r = cur_r + 1;
+      sampling = m.sampling;
+      acc_reset(A);
+      return true;
+    };
 
     // Sub-tiles are dealt round-robin: warp w takes w, w + NW, w + 2 NW, ...
+    // The four sub-tiles of a tile go to four warps that also share every
+    // tile k +- 3 NW / kSubPerStage ...; a warp has consumed the stage's
+    // previous tile (k - kStages) itself before it waits for tile k, so the
+    // parity of the stage's full barrier is unambiguous, and once it has
+    // completed the tile's description and header are in place.
     for (int u = warp; u < n_sub; u += NW) {
       if (*(volatile int*)&ctrl->abort) break;
       const int k = u / Sh::kSubPerStage;
       const int sub = u & (Sh::kSubPerStage - 1);
       const int st = k % kStages;
-      // A warp may run up to a few sub-tiles ahead of the ring, past the
-      // stage's current phase; the parity of the full barrier is only
-      // unambiguous once the producer has issued tile k (which it does after
-      // the stage's previous tile, k - kStages, was released).  The row
-      // change (and its deposits) is handled before the stage is waited for,
-      // so a warp never holds a stage while it waits for a row slot.
-      if (!wait_counter_above(&ctrl->issued, k, a.wait_ns)) {
-        fail = true;
-        break;
-      }
-      const TileMeta m = meta[st];
-      if (m.r != cur_r) {
-        if (cur_r >= 0 && !deposit(cur_r, false)) {
-          fail = true;
-          break;
-        }
-        if (cur_r >= 0) next_r = cur_r + 1;
-        if (!owe_empty(m.r)) {
-          fail = true;
-          break;
-        }
-        cur_r = m.r;
-        next_r = cur_r + 1;
-        sampling = m.sampling;
-        acc_reset(A);
-      }
       if (!mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u, a.wait_ns)) {
         fail = true;
         break;
       }
+      const TileMeta m = meta[st];
       const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
       const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
       const uint32_t* wd = words + st * Sh::kStageGroups;
@@ -783,13 +901,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       const bool fast =
           __all_sync(0xffffffffu, a.vec_ok && (!has0 || len0 == kGroup) && (!has1 || len1 == kGroup));
       uint32_t x0 = 0, x1 = 0;
-      if (sampling) {
+      if (m.sampling) {
         if (has0) x0 = wd[gl0];
         if (has1) x1 = wd[gl1];
       }
-      // The lane's step for group j with maximum mg: a new maximum makes it
-      // the lane's top group (exact form); otherwise its sums join the rest
-      // (term by term when the vector sums are not finite: -inf logits).
       // The lane's step for group j with maximum mg: a new maximum makes it
       // the lane's top group; otherwise its sums join the rest.
       // sums(ref, S, W): the group's sums relative to ref.
@@ -809,12 +924,18 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         if (sampling) lane_race(A, Z, x, j);
       };
       if (DT == kBF16 && fast && any) {
-        // both groups into registers, then the stage goes back to the producer
+        // both groups into registers, then the stage goes back to the
+        // producer; the row change (which may wait for a row slot) comes
+        // after the release
         uint32_t G0[32], G1[32];
         load_group_bf16(sbase + (size_t)(has0 ? gl0 : 0) * 128, rot, G0);
         load_group_bf16(sbase + (size_t)(has1 ? gl1 : has0 ? gl0 : 0) * 128, rot, G1);
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[st]);
+        if (!enter_row(m)) {
+          fail = true;
+          break;
+        }
         if (has0)
           fold(group_max_bf16(G0), j0, x0, [&](float ref, float& S, float& W) {
             group_sums_bf16(G0, a.c2, ref, S, W);
@@ -826,6 +947,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
             if (!(W >= -3.0e38f && S <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S, W);
           });
         continue;
+      }
+      if (!enter_row(m)) {
+        fail = true;
+        break;
       }
       if (any) {
         auto group = [&](bool has, int gl, int len, int j, uint32_t x) {
@@ -862,18 +987,62 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     }
   }
 
-  __syncthreads();
+  // Every warp reaches the block barrier converged (the copy producer's lane
+  // 0 leaves its loop long after lanes 1-31).
+  block_sync();
   // After an abort, wait (bounded) for bulk copies still in flight into this
   // CTA's shared memory before it may exit.  Every role has left its loop, so
   // the issued count is final: first make the second arrival of every issued
   // tile the word producer did not reach, so each stage's last phase can
   // complete once its copy lands.
-  if (tid == 0 && *(volatile int*)&ctrl->abort) {
+  const bool aborted = *(volatile int*)&ctrl->abort != 0;
+  if (tid == 0 && aborted) {
     const int issued = ld_acquire_shared(&ctrl->issued);
     for (int k = ctrl->words_arrived; k < issued; ++k) mbar_arrive(&full[k % kStages]);
     for (int st = 0; st < kStages && st < issued; ++st) {
       const int n2 = (issued - st + kStages - 1) / kStages;
       mbar_wait(&full[st], (uint32_t)(n2 - 1) & 1u, kDrainLimitNs);
+    }
+  }
+  if (!a.run_epilogue) return;
+  // The decisions of the canvases this CTA completed, with every thread and
+  // the ring's shared memory; they write stop flags, so first every CTA of
+  // the grid must have read them (the started counter).
+  const int n_epi = ctrl->n_epi;
+  if (n_epi > 0 && !aborted) {
+    if (tid == 0 && !ctrl->epi_ok) {
+      const uint64_t t0 = global_ns();
+      bool ok = true;
+      while (ld_acquire_gpu(a.sync_cnt) < (int)gridDim.x) {
+        if (global_ns() - t0 > a.wait_ns) {
+          ok = false;
+          break;
+        }
+        __nanosleep(64);
+      }
+      if (!ok) atomicOr(a.status, kStatusTimeout);
+      ctrl->epi_ok = ok;
+    }
+    block_sync();
+    if (ctrl->epi_ok) {
+      const EpiSmem m = epi_smem(ring, a.L);
+      for (int e = 0; e < n_epi; ++e) {
+        const int bi = epi[e];
+        epi_load_state<Sh::kThreads>(a, bi, m);
+        epi_load_rows<Sh::kThreads>(a, bi, m);
+        block_sync();
+        canvas_epilogue<Sh::kThreads>(a, bi, m);
+        if (tid == 0) a.canvas_cnt[bi] = 0;  // zero again for the next step
+        block_sync();
+      }
+    }
+  }
+  // the last CTA to leave zeroes the grid counters for the next step
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(a.sync_cnt + 1, 1) == (int)gridDim.x - 1) {
+      a.sync_cnt[0] = 0;
+      a.sync_cnt[1] = 0;
     }
   }
 }

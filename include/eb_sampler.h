@@ -152,7 +152,10 @@ int eb_sampler_init(eb_sampler_t** out, const eb_config_t* cfg, int device);
 int eb_sampler_init_canvas(eb_sampler_t* h, int32_t* canvas, uint8_t* committed,
                            uint8_t* stop_flags, void* stream);
 
-/* One denoising step `step` (0 .. num_steps-1) on `stream`.  `step` must be
+/* One denoising step `step` (0 .. num_steps-1) on `stream`: one kernel,
+   launched as a programmatic dependent of the stream's previous kernel
+   (its shared-memory set-up overlaps that kernel's end; it reads nothing
+   before that kernel has completed).  `step` must be
    0 (which restarts the step sequence) or the previous step + 1, else
    EB_ERR_STEP_ORDER.  Canvases whose stop flag is set are skipped: their
    logits are not read and their buffers are left untouched.  For every
@@ -262,12 +265,11 @@ size_t eb_slice_record_bytes(void);
 
 /* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
    the caller) is non-NULL, every following eb_sampler_step records it on
-   its stream between the step's two kernels (the stream pass and the canvas
-   epilogue), so that the caller can time them apart with events recorded
-   before and after the call.  Recording it keeps the second kernel from
-   starting early (programmatic dependent launch), so set it only for
-   timing; NULL turns it off.  No counterpart in the method: it measures the
-   implementation. */
+   its stream right after the step's kernel, so that the caller can time that
+   kernel with an event recorded before the call.  Recording it keeps the
+   next kernel on the stream from starting early (programmatic dependent
+   launch), so set it only for timing; NULL turns it off.  No counterpart in
+   the method: it measures the implementation. */
 int eb_sampler_set_split_event(eb_sampler_t* h, void* event);
 
 /* Diagnostic hook: the limit, in nanoseconds, of every wait of the stream
