@@ -15,10 +15,11 @@ Timing: W eager warm-up steps, then timed regions of exactly K steps, each
 with CUDA events on the launching stream between a barrier + synchronize on
 both sides (max over ranks); the K steps are replayed from CUDA graphs (one
 per full 48-step trajectory, one for the remaining prefix; each starts with
-the canvas init kernel), and the median over the regions is reported.  The
-kernels' own launch durations (for the roofline) come from per-launch events
-over one eager trajectory.  For N > 1 each rank runs its own canvas (global
-canvas index = rank): no data-path collective, weak scaling.
+the canvas init kernel), and the median over the regions is reported.  A
+step is one kernel launch, so the step kernel's average launch duration (for
+the roofline) is the region's time over its K launches.  For N > 1 each rank
+runs its own canvas (global canvas index = rank): no data-path collective,
+weak scaling.
 
 At N = 1 the other large workloads (serve 8x, br 4x, stress 32x fp32) are
 timed afterwards as whole 48-step trajectories and reported under "configs".
@@ -312,26 +313,6 @@ class Trajectory:
             self.graphs[n] = g
         return self.graphs[n]
 
-    def kernel_times(self):
-        """Mean per-launch durations (ms) of the step's two kernels over one
-        eager trajectory (steps with an active canvas, step 0 excluded):
-        events before the step, between its kernels (the library's split
-        event) and after it, all on the launching stream."""
-        import torch
-        stream = torch.cuda.current_stream(self.dev)
-        evs = []
-        self.eb.init_canvas(self.canvas, self.committed, self.stop)
-        for s in range(self.N):
-            a, m, b = (torch.cuda.Event(enable_timing=True) for _ in range(3))
-            self.eb.set_split_event(m)
-            a.record(stream)
-            self.eb.step(self.lg(s), s, self.canvas, self.committed, self.H, self.amax, self.stop)
-            b.record(stream)
-            evs.append((s, a, m, b))
-        self.eb.set_split_event(None)
-        torch.cuda.synchronize()
-        return evs
-
     def close(self):
         self.graphs.clear()
         self.eb.close()
@@ -356,25 +337,21 @@ def timed_regions(replay, repeats, barrier, stream):
     return out
 
 
-def roofline_of(tr, active, peak, peak_kind):
-    """Stream-kernel roofline of a workload: algorithmic bytes per launch
-    (every logit of the active canvases once) over its event-timed duration."""
-    evs = tr.kernel_times()
-    w = tr.w
-    ks, fs, byts = [], [], []
-    for s, a, m, b in evs:
-        if s == 0 or not active[s]:
-            continue
-        ks.append(a.elapsed_time(m))
-        fs.append(m.elapsed_time(b))
-        byts.append(active[s] * w.L * w.V * w.elt)
-    k_ms = statistics.mean(ks)
-    bytes_launch = statistics.mean(byts)
+def roofline_of(kernel, launches, bytes_total, region_ms, peak, peak_kind):
+    """Step-kernel roofline of a timed region.  A step is one kernel launch
+    (the stream kernel, canvas decisions included), so its average launch
+    duration is the region's time over the launches in it; the region's few
+    canvas-init launches (about 2 us each) are counted against it.
+    Algorithmic bytes per launch: every logit of the canvases active at that
+    step, once."""
+    k_ms = region_ms / launches
+    bytes_launch = bytes_total / launches
     achieved = bytes_launch / (k_ms * 1e-3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-            "frac": achieved / peak, "kernel": f"ebk::stream_kernel<{'f32' if w.elt == 4 else 'bf16'}>",
-            "kernel_ms": k_ms, "finish_kernel_ms": statistics.mean(fs),
+            "frac": achieved / peak, "kernel": kernel, "kernel_ms": k_ms,
             "algorithmic_bytes": bytes_launch,
+            "timing": "CUDA events around graph replays on the launching stream; "
+                      "region time / step-kernel launches",
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"}
 
 
@@ -475,7 +452,8 @@ def run_ours(args):
         if g_rem is not None:
             g_rem.replay()
 
-    launches = full * (2 * N + 1) + ((2 * rem + 1) if rem else 0)
+    # one kernel per step, one init kernel per graph
+    launches = full * (N + 1) + ((rem + 1) if rem else 0)
     positions = full * sum(active) * w.L + sum(active[:rem]) * w.L
     bytes_total = (full * sum(active) + sum(active[:rem])) * w.L * w.V * w.elt
     repeats = args.repeats or max(3, min(50, int(0.5 / max(1e-5, K * 40e-6))))
@@ -498,7 +476,8 @@ def run_ours(args):
         traj = timed_regions(g48.replay, 3, barrier, stream)
         traj_ms = max_over_ranks(statistics.median(traj)) / N
 
-    roof = roofline_of(tr, active, peak, peak_kind)
+    kname = f"ebk::stream_kernel<{'f32' if w.elt == 4 else 'bf16'}>"
+    roof = roofline_of(kname, K, bytes_total, el_ms, peak, peak_kind)
     roof["traffic"] = recorded_traffic()
 
     # end-to-end: host (pinned) logits -> device, step, result back to host, every step
@@ -560,15 +539,14 @@ def run_ours(args):
         ms = max_over_ranks(statistics.median(tx_times))
         pos = sum_over_ranks(float(sum(act) * wx.L))
         byt = sum_over_ranks(float(sum(act) * wx.L * wx.V * wx.elt))
-        rf = roofline_of(tx, act, peak, peak_kind)
+        rf = roofline_of("", wx.num_steps, sum(act) * wx.L * wx.V * wx.elt, ms, peak, peak_kind)
         gbs = byt / (ms * 1e-3) / 1e9
         extra[name] = {
             "workload": desc, "value": pos / (ms * 1e-3), "unit": UNIT,
             "ms_per_step": ms / wx.num_steps, "steps": wx.num_steps, "repeats": len(tx_times),
             "active_canvases_per_step": act, "dtype": "f32" if wx.elt == 4 else "bf16",
             "hbm_gbs": gbs, "hbm_frac_of_peak": gbs / (peak * world),
-            "roofline": {k: rf[k] for k in ("achieved", "frac", "kernel_ms", "finish_kernel_ms",
-                                            "algorithmic_bytes")},
+            "roofline": {k: rf[k] for k in ("achieved", "frac", "kernel_ms", "algorithmic_bytes")},
         }
         tx.close()
         del tx, gx

@@ -330,6 +330,36 @@ __device__ __forceinline__ void group_sums_bf16(const uint32_t (&A)[32], float c
   W = sum4(w);
 }
 
+// The sums of two groups relative to one reference, interleaved word by
+// word: twice the independent exponentials in flight of one group's loop.
+// Per group, the same terms and rules as group_sums_bf16.
+__device__ __forceinline__ void group_sums2_bf16(const uint32_t (&A)[32], const uint32_t (&B)[32],
+                                                 float c2, float ref, float& SA, float& WA,
+                                                 float& SB, float& WB) {
+  const float2 c2v = make_float2(c2, c2);
+  const float2 nrc = make_float2(-ref * c2, -ref * c2);
+  float2 sa[2], wa[2], sb[2], wb[2];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) sa[i] = wa[i] = sb[i] = wb[i] = make_float2(0.f, 0.f);
+#pragma unroll
+  for (int q = 0; q < 32; ++q) {
+    const float2 za = make_float2(bf16_lo(A[q]), bf16_hi(A[q]));
+    const float2 zb = make_float2(bf16_lo(B[q]), bf16_hi(B[q]));
+    const float2 da = ffma2(za, c2v, nrc);
+    const float2 db = ffma2(zb, c2v, nrc);
+    const float2 pa = make_float2(ex2(da.x), ex2(da.y));
+    const float2 pb = make_float2(ex2(db.x), ex2(db.y));
+    sa[q & 1] = fadd2(sa[q & 1], pa);
+    wa[q & 1] = ffma2(pa, da, wa[q & 1]);
+    sb[q & 1] = fadd2(sb[q & 1], pb);
+    wb[q & 1] = ffma2(pb, db, wb[q & 1]);
+  }
+  SA = (sa[0].x + sa[0].y) + (sa[1].x + sa[1].y);
+  WA = (wa[0].x + wa[0].y) + (wa[1].x + wa[1].y);
+  SB = (sb[0].x + sb[0].y) + (sb[1].x + sb[1].y);
+  WB = (wb[0].x + wb[0].y) + (wb[1].x + wb[1].y);
+}
+
 // Exact form of a group relative to ref >= every element: n = elements equal
 // to ref, amin = the lowest of them (kNone if none), S and W over the
 // others with d = (z - ref) c2 (the difference is exact for bf16 values of

@@ -936,16 +936,43 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           fail = true;
           break;
         }
-        if (has0)
-          fold(group_max_bf16(G0), j0, x0, [&](float ref, float& S, float& W) {
-            group_sums_bf16(G0, a.c2, ref, S, W);
-            if (!(W >= -3.0e38f && S <= 3.0e38f)) group_sums_bf16<true>(G0, a.c2, ref, S, W);
-          });
-        if (has1)
-          fold(group_max_bf16(G1), j1, x1, [&](float ref, float& S, float& W) {
-            group_sums_bf16(G1, a.c2, ref, S, W);
-            if (!(W >= -3.0e38f && S <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S, W);
-          });
+        // Both groups against one reference, the larger of the lane's
+        // maximum and theirs: a group raising it becomes the top group (the
+        // first on equal maxima), the other joins the rest; then the race,
+        // group 0 first.
+        const float mg0 = has0 ? group_max_bf16(G0) : -INFINITY;
+        const float mg1 = has1 ? group_max_bf16(G1) : -INFINITY;
+        const bool v0 = mg0 > -INFINITY, v1 = mg1 > -INFINITY;  // not every logit -inf
+        if (!(v0 || v1)) continue;
+        const float mg = fmaxf(mg0, mg1);
+        const bool new_top = mg > A.M;
+        const float ref = new_top ? mg : A.M;
+        float S0, W0, S1, W1;
+        group_sums2_bf16(G0, G1, a.c2, ref, S0, W0, S1, W1);
+        if (v0 && !(W0 >= -3.0e38f && S0 <= 3.0e38f)) group_sums_bf16<true>(G0, a.c2, ref, S0, W0);
+        if (v1 && !(W1 >= -3.0e38f && S1 <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S1, W1);
+        if (new_top) {
+          const bool top0 = mg0 == mg;
+          lane_new_top(A, mg, top0 ? j0 : j1, top0 ? S0 : S1, top0 ? W0 : W1, a.c2);
+          const bool rest = top0 ? v1 : v0;
+          if (rest) {
+            A.Sr += top0 ? S1 : S0;
+            A.Wr += top0 ? W1 : W0;
+          }
+        } else {
+          if (v0) {
+            A.Sr += S0;
+            A.Wr += W0;
+          }
+          if (v1) {
+            A.Sr += S1;
+            A.Wr += W1;
+          }
+        }
+        if (sampling) {
+          if (v0) lane_race(A, S0, x0, j0);
+          if (v1) lane_race(A, S1, x1, j1);
+        }
         continue;
       }
       if (!enter_row(m)) {

@@ -297,7 +297,7 @@ def test_slice_handle_refuses_the_plain_step(E):
     h.close()
 
 
-def test_split_event_times_the_two_kernels(E):
+def test_split_event_is_recorded_after_the_step_kernel(E):
     w = MID.replace(B=1, num_steps=4)
     eb = make_sampler(E, w)
     canvas, committed, stop = eb.new_canvas()
@@ -314,7 +314,7 @@ def test_split_event_times_the_two_kernels(E):
         b.record()
         torch.cuda.synchronize()
         if use:
-            assert a.elapsed_time(m) > 0 and m.elapsed_time(b) > 0
+            assert a.elapsed_time(m) > 0 and m.elapsed_time(b) >= 0
             assert torch.equal(H, H0)  # recording the event changes no result
         H0 = H.clone()
     eb.set_split_event(None)
