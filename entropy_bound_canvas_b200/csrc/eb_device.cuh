@@ -165,11 +165,21 @@ __device__ __forceinline__ int ld_acquire_shared(const int* p) {
 }
 
 // Global counter read with acquire semantics at GPU scope (pairs with a
-// writer's fence before its atomic update).
+// writer's release update).
 __device__ __forceinline__ int ld_acquire_gpu(const int* p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+// Atomic add at GPU scope with acquire-release semantics: this thread's
+// earlier writes are visible to whoever observes the new value, and the
+// writes of those whose additions this one observes are visible to it.
+// Returns the old value.
+__device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
+  return old;
 }
 
 // Waits (bounded like mbar_wait) until *p > k.

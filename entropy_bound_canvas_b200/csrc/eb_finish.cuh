@@ -467,16 +467,28 @@ __device__ __forceinline__ void epi_load_state(const StepArgs& a, int bi, const 
   if (threadIdx.x == 0) m.ctrl->stable_prev = a.stable[bi];
 }
 
-// This step's per-position results of canvas bi, written by other CTAs
-// (read through L2).
+// What the previous step left and this step's per-position results of
+// canvas bi (written by other CTAs: read through L2), all of a position's
+// loads issued before its shared-memory stores.
 template <int NT>
-__device__ __forceinline__ void epi_load_rows(const StepArgs& a, int bi, const EpiSmem& m) {
+__device__ __forceinline__ void epi_load(const StepArgs& a, int bi, const EpiSmem& m) {
   const size_t row0 = (size_t)bi * (size_t)a.L;
+  if (threadIdx.x == 0) m.ctrl->stable_prev = a.stable[bi];
   for (int l = threadIdx.x; l < a.L; l += NT) {
-    m.H[l] = __ldcg(a.H_out + row0 + l);
-    m.am[l] = __ldcg(a.amax_out + row0 + l);
-    m.smp[l] = __ldcg(a.sample + row0 + l);
-    m.pm[l] = __ldcg(a.pmax + row0 + l);
+    const int prev = a.prev_amax[row0 + l];
+    const int tok = a.canvas[row0 + l];
+    const uint8_t cm = a.committed[row0 + l];
+    const float H = __ldcg(a.H_out + row0 + l);
+    const int am = __ldcg(a.amax_out + row0 + l);
+    const int smp = __ldcg(a.sample + row0 + l);
+    const float pm = __ldcg(a.pmax + row0 + l);
+    m.prev[l] = prev;
+    m.tok[l] = tok;
+    m.open[l] = cm == 0;
+    m.H[l] = H;
+    m.am[l] = am;
+    m.smp[l] = smp;
+    m.pm[l] = pm;
   }
 }
 

@@ -772,17 +772,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           sp.nseg > 1 && __shfl_sync(0xffffffffu, pre, 0) == sp.nseg - 1;
       Rec other;
       other.M = -INFINITY;
+      __syncwarp();  // lane 0's acquire before the other lanes' record loads
       if (others_done && lane < sp.nseg && lane != sp.seg) other = ld_rec(rr + lane);
       const Rec own = part_finalize(a, mine, pl, bi, l);
       // the canvas's finished positions; the CTA finishing its last one runs
       // the canvas's decisions after its roles are done
       auto count_canvas = [&]() {
         if (!a.run_epilogue || lane != 0) return;
-        __threadfence();
-        if (atomicAdd(a.canvas_cnt + bi, 1) == a.L - 1) {
-          __threadfence();
+        if (atom_add_acq_rel_gpu(a.canvas_cnt + bi, 1) == a.L - 1)
           epi[atomicAdd(&ctrl->n_epi, 1)] = (uint16_t)bi;
-        }
       };
       if (sp.nseg == 1) {
         const RowFinal F = combine_records(1, [&](int) { return own; }, a.c2);
@@ -795,12 +793,11 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         int old = 0;
         if (lane == 0) {
           rr[sp.seg] = own;
-          __threadfence();
-          old = atomicAdd(a.row_cnt + grow, 1);
+          old = atom_add_acq_rel_gpu(a.row_cnt + grow, 1);
         }
         last = __shfl_sync(0xffffffffu, old, 0) == sp.nseg - 1;
         if (!last) continue;
-        __threadfence();
+        __syncwarp();  // lane 0's acquire before the other lanes' record loads
         if (lane < sp.nseg && lane != sp.seg) other = ld_rec(rr + lane);
       }
       auto rec = [&](int i) -> Rec {
@@ -1055,8 +1052,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       const EpiSmem m = epi_smem(ring, a.L);
       for (int e = 0; e < n_epi; ++e) {
         const int bi = epi[e];
-        epi_load_state<Sh::kThreads>(a, bi, m);
-        epi_load_rows<Sh::kThreads>(a, bi, m);
+        epi_load<Sh::kThreads>(a, bi, m);
         block_sync();
         canvas_epilogue<Sh::kThreads>(a, bi, m);
         if (tid == 0) a.canvas_cnt[bi] = 0;  // zero again for the next step
