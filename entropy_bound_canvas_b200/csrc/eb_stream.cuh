@@ -83,7 +83,8 @@ struct StreamCtrl {
   int words_arrived;  // tiles whose second (header) arrival was made
   int n_epi;          // canvases whose decisions this CTA runs
   int epi_ok;         // every CTA of the grid has read the stop flags
-  int wcnt[32];
+  int ready;          // the producer has published act, n_sub
+  int nread;          // warps that have read the stop flags
 };
 
 // What the producer tells the consumers about the tile in a stage.
@@ -202,26 +203,25 @@ __device__ __forceinline__ int count_tiles(unsigned long long lo, unsigned long 
   return n;
 }
 
-// Active canvases in index order, from the stop flags as they were when the
-// step began (only the epilogue kernel, after this one, writes them).
-__device__ __forceinline__ int build_active_list(const uint8_t* stop_flags, int B, uint16_t* act,
-                                                 int* wcnt, int nthreads) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int nwarps = nthreads / 32;
-  int base = 0;
-  for (int b0 = 0; b0 < B; b0 += nthreads) {
-    const int b = b0 + tid;
+// Active canvases (stop flag clear) counted by one warp from the stop flags
+// as they were when the step began (only this kernel's canvas decisions, at
+// its end, write them); with act != nullptr the warp also lists them in index
+// order, and with act_index != nullptr writes every canvas's place in that
+// list (-1: stopped).
+__device__ __forceinline__ int warp_active_list(const uint8_t* stop_flags, int B, uint16_t* act,
+                                                int32_t* act_index) {
+  const int lane = threadIdx.x & 31;
+  int n = 0;
+  for (int b0 = 0; b0 < B; b0 += 32) {
+    const int b = b0 + lane;
     const bool on = b < B && __ldcg(stop_flags + b) == 0;
     const unsigned bal = __ballot_sync(0xffffffffu, on);
-    if (lane == 0) wcnt[warp] = __popc(bal);
-    block_sync();
-    int off = base;
-    for (int w = 0; w < warp; ++w) off += wcnt[w];
-    if (on) act[off + __popc(bal & ((1u << lane) - 1u))] = (uint16_t)b;
-    for (int w = 0; w < nwarps; ++w) base += wcnt[w];
-    block_sync();
+    const int rank = n + __popc(bal & ((1u << lane) - 1u));
+    if (on && act != nullptr) act[rank] = (uint16_t)b;
+    if (b < B && act_index != nullptr) act_index[b] = on ? rank : -1;
+    n += __popc(bal);
   }
-  return base;
+  return n;
 }
 
 // Where row r's records live: the stream CTAs that own part of it are
@@ -547,35 +547,52 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     ctrl->words_arrived = 0;
     ctrl->n_epi = 0;
     ctrl->epi_ok = 0;
+    ctrl->ready = 0;
+    ctrl->nread = 0;
     for (int i = 0; i < kSlots; ++i) {
       slots[i].q = i;
       slots[i].count = 0;
     }
     fence_mbar_init();
   }
+  // Barriers and slots initialized before any warp uses them.
+  block_sync();
   // Everything above is this CTA's own shared memory; from here on the
   // kernel reads what the previous step's kernel wrote (stop flags, canvas
-  // state, counters): wait until that grid has completed.
+  // state, counters): wait until that grid has completed.  The next kernel
+  // on the stream may be scheduled from now on, wherever an SM has room: it
+  // waits for this grid's completion in turn before reading anything this
+  // grid writes.
   griddep_wait();
-  const int n_act = build_active_list(a.stop_flags, a.B, act, ctrl->wcnt, Sh::kThreads);
-  if (a.run_epilogue && tid == 0) atomicAdd(a.sync_cnt, 1);  // this CTA has read the stop flags
-  if (blockIdx.x == 0) {  // publish the active list for the epilogue kernel
-    for (int b = tid; b < a.B; b += Sh::kThreads) a.act_index[b] = -1;
-    block_sync();
-    for (int i = tid; i < n_act; i += Sh::kThreads) a.act_index[act[i]] = i;
-    if (tid == 0) *a.n_act = n_act;
+  griddep_launch_dependents();
+  // Every warp counts the active canvases itself (no block barrier); the
+  // producer warp also lists them for the others (published with `ready`),
+  // and in block 0 writes the list's index for the split-vocabulary combine.
+  const int n_act = warp_active_list(
+      a.stop_flags, a.B, warp == NW ? act : nullptr,
+      (warp == NW && blockIdx.x == 0) ? a.act_index : nullptr);
+  if (lane == 0) {
+    if (warp == NW && blockIdx.x == 0) *a.n_act = n_act;
+    // the last warp of the CTA to have read the stop flags says so
+    if (atomicAdd(&ctrl->nread, 1) == Sh::kThreads / 32 - 1 && a.run_epilogue)
+      atomicAdd(a.sync_cnt, 1);
   }
   const int G = gridDim.x;
   const unsigned long long NG =
       (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
   const unsigned long long g_lo = range_start(blockIdx.x, NG, G);
   const unsigned long long g_hi = range_start(blockIdx.x + 1, NG, G);
-  if (tid == 0) ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
-  block_sync();
-  // The next kernel on the stream may be scheduled from now on, wherever an
-  // SM has room: it waits for this grid's completion (griddepcontrol.wait)
-  // before reading anything this grid writes.
-  griddep_launch_dependents();
+  // The other roles start once the producer has published the active list
+  // and the range's sub-tile count (right after its first copy).
+  auto wait_ready = [&]() -> bool {
+    int ok = 1;
+    if (lane == 0 && !wait_counter_above(&ctrl->ready, 0, a.wait_ns)) {
+      atomicOr(a.status, kStatusTimeout);
+      *(volatile int*)&ctrl->abort = 1;
+      ok = 0;
+    }
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+  };
 
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
   const char* logits = reinterpret_cast<const char*>(a.logits);
@@ -592,8 +609,16 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // ------------------------------------------------------- copy producer
     // Lane 0 alone: waits for a free stage, issues the tile's bulk copy (the
     // stage's first arrival, with the bytes) and writes its description.  No
-    // global load ever delays the next copy.
+    // global load ever delays the next copy.  Right after its first copy it
+    // publishes the range's sub-tile count and the active list (`ready`).
+    __syncwarp();  // the warp's active list before lane 0 publishes it
     if (lane == 0) {
+      bool published = false;
+      auto publish = [&]() {
+        ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
+        st_release_shared(&ctrl->ready, 1);
+        published = true;
+      };
       // Logits are read once: L2 evict-first, so that the stream does not push
       // out the kernel's code and small state.
       const uint64_t policy = evict_first_policy();
@@ -638,12 +663,14 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         m.pad = 0;
         meta[st] = m;
         st_release_shared(&ctrl->issued, k + 1);
+        if (!published) publish();
         ++k;
         if (++st == kStages) {
           st = 0;
           ph ^= 1u;
         }
       }
+      if (!published) publish();
       // Have all CTAs of the grid read the stop flags?  (Checked here, long
       // before this CTA can need it, so that a canvas's decisions at the end
       // rarely wait for the round trip.)
@@ -656,7 +683,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // group-stream Philox words of a drawing position's groups into the
     // stage's header and makes the stage's second arrival.  The committed
     // flags of the range's first 32 rows are loaded at once, at the start.
-    const int n_tiles = ctrl->n_sub / Sh::kSubPerStage;
+    const int n_tiles = wait_ready() ? ctrl->n_sub / Sh::kSubPerStage : 0;
     uint32_t open_bits = 0;
     if (!a.greedy) {
       const long long r = r_first + lane;
@@ -715,7 +742,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // Finisher f takes the rows q = f, f + kFinishers, ... of the range, so
     // that rows completed close together (at the end of the range) are
     // finished in parallel.
-    const int nrows = (int)(r_end - r_first);
+    const int nrows = wait_ready() ? (int)(r_end - r_first) : 0;
     const int f = warp - (NW + 2);
     for (int q = f; q < nrows; q += Sh::kFinishers) {
       RowSlot* sl = &slots[q % kSlots];
@@ -812,7 +839,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     }
   } else {
     // ------------------------------------------------------------ consumers
-    const int n_sub = ctrl->n_sub;
+    const int n_sub = wait_ready() ? ctrl->n_sub : 0;
     long long cur_r = -1;
     long long next_r = r_first;  // first row of the range this warp still owes a deposit
     int sampling = 0;
