@@ -1087,10 +1087,11 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       }
     }
   }
-  // the last CTA to leave zeroes the grid counters for the next step
+  // The last CTA to leave zeroes the grid counters for the next step (the
+  // release orders this CTA's reads of them before its count; the acquire,
+  // everyone's before the reset).
   if (tid == 0) {
-    __threadfence();
-    if (atomicAdd(a.sync_cnt + 1, 1) == (int)gridDim.x - 1) {
+    if (atom_add_acq_rel_gpu(a.sync_cnt + 1, 1) == (int)gridDim.x - 1) {
       a.sync_cnt[0] = 0;
       a.sync_cnt[1] = 0;
     }
