@@ -142,14 +142,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
 
+// Gives up (false) after limit_ns, or once *abort is set when abort is given
+// (checked only on the slow path).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint64_t limit_ns = kWaitLimitNs) {
+                                          uint64_t limit_ns = kWaitLimitNs,
+                                          const int* abort = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
 #pragma unroll 1
     for (int i = 0; i < 32; ++i)
       if (mbar_try_wait(bar, parity)) return true;
+    if (abort != nullptr && *(const volatile int*)abort) return false;
     if (global_ns() - t0 > limit_ns) return false;
   }
 }

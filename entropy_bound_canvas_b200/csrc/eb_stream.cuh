@@ -96,7 +96,7 @@ struct TileMeta {
   int l;         // position
   int sampling;  // open position of a sampled (not greedy) run
   int delta;     // byte offset of the tile's first logit in the stage
-  int pad;
+  int whole;     // every group whole and 16-byte aligned: the vector path
 };
 
 // A row slot: the consumer warps' deposits for one row of the CTA's range.
@@ -660,7 +660,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         m.l = t.l;
         m.sampling = 0;  // set by the word producer
         m.delta = (int)(reinterpret_cast<uintptr_t>(src) - a0);
-        m.pad = 0;
+        m.whole = a.vec_ok && (t.j0 + t.cnt) * kGroup <= a.V;
         meta[st] = m;
         st_release_shared(&ctrl->issued, k + 1);
         if (!published) publish();
@@ -904,11 +904,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // parity of the stage's full barrier is unambiguous, and once it has
     // completed the tile's description and header are in place.
     for (int u = warp; u < n_sub; u += NW) {
-      if (*(volatile int*)&ctrl->abort) break;
       const int k = u / Sh::kSubPerStage;
       const int sub = u & (Sh::kSubPerStage - 1);
       const int st = k % kStages;
-      if (!mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u, a.wait_ns)) {
+      if (!mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u, a.wait_ns, &ctrl->abort)) {
         fail = true;
         break;
       }
@@ -919,11 +918,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       const bool any = sub * Sh::kSubGroups < m.cnt;  // warp-uniform
       const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
       const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
-      const int len0 = has0 ? min(kGroup, a.V - j0 * kGroup) : 0;
-      const int len1 = has1 ? min(kGroup, a.V - j1 * kGroup) : 0;
-      // whole 16-byte-aligned groups (or none) in every lane: the vector path
-      const bool fast =
-          __all_sync(0xffffffffu, a.vec_ok && (!has0 || len0 == kGroup) && (!has1 || len1 == kGroup));
+      // whole 16-byte-aligned groups in the whole tile: the vector path
+      const bool fast = m.whole != 0;
       uint32_t x0 = 0, x1 = 0;
       if (m.sampling) {
         if (has0) x0 = wd[gl0];
@@ -1019,6 +1015,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
                  W = e.W;
                });
         };
+        const int len0 = has0 ? min(kGroup, a.V - j0 * kGroup) : 0;
+        const int len1 = has1 ? min(kGroup, a.V - j1 * kGroup) : 0;
         group(has0, gl0, len0, j0, x0);
         group(has1, gl1, len1, j1, x1);
       }
