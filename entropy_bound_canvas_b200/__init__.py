@@ -102,6 +102,12 @@ def _lib():
         L.eb_strerror.restype = C.c_char_p
         L.eb_version.argtypes = []
         L.eb_version.restype = i32
+        L.eb_lmhead_logits.argtypes = [vp, vp, i32, i32, i32, vp, vp]
+        L.eb_lmhead_logits.restype = i32
+        L.eb_lmhead_reserve.argtypes = [vp, i32]
+        L.eb_lmhead_reserve.restype = i32
+        L.eb_lmhead_step.argtypes = [vp, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.eb_lmhead_step.restype = i32
         _LIB = L
     return _LIB
 
@@ -134,6 +140,27 @@ def _check(rc: int, what: str):
 def _torch():
     import torch
     return torch
+
+
+def lmhead_logits(hidden, weight, out=None):
+    """The LM head's logits hidden @ weight^T (bf16 [rows, d] and [V, d] on
+    one device) formed by the fused LM-head kernel's tensor-core contraction,
+    written as fp32 [rows, V]: the diagnostic form of eb_lmhead_step."""
+    torch = _torch()
+    for t, n in ((hidden, "hidden"), (weight, "weight")):
+        if t.dtype != torch.bfloat16 or t.dim() != 2 or not t.is_contiguous():
+            raise ValueError(f"{n} must be a contiguous 2-D bf16 tensor")
+    rows, d = hidden.shape
+    V = weight.shape[0]
+    if weight.shape[1] != d:
+        raise ValueError("hidden and weight disagree on the hidden size")
+    if out is None:
+        out = torch.empty((rows, V), dtype=torch.float32, device=hidden.device)
+    stream = torch.cuda.current_stream(hidden.device).cuda_stream
+    _check(_lib().eb_lmhead_logits(C.c_void_p(hidden.data_ptr()), C.c_void_p(weight.data_ptr()),
+                                   int(rows), int(V), int(d), C.c_void_p(out.data_ptr()),
+                                   C.c_void_p(stream)), "eb_lmhead_logits")
+    return out
 
 
 def shard_canvases(B: int, world: int, rank: int):
@@ -221,6 +248,31 @@ class EBSampler:
             self._ptr(argmax, torch.int32, (self.B, self.L), "argmax"),
             self._ptr(stop_flags, torch.uint8, (self.B,), "stop_flags"), self._stream()),
             "eb_sampler_step")
+
+    # -- the sampler fused into the LM head --------------------------------------
+    def lmhead_step(self, hidden, weight, step: int, canvas, committed, entropies, argmax,
+                    stop_flags):
+        """A step from the decoder's hidden states: hidden [B, L, d] (or
+        [B*L, d]) and the LM head weight [V, d], both bf16; the logits are
+        formed on the tensor cores and reduced on chip (never written)."""
+        torch = _torch()
+        for t, n in ((hidden, "hidden"), (weight, "weight")):
+            if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.device != self.device:
+                raise ValueError(f"{n} must be a contiguous bf16 tensor on {self.device}")
+        d = int(hidden.shape[-1])
+        if hidden.numel() != self.B * self.L * d or tuple(weight.shape) != (self.V, d):
+            raise ValueError(f"hidden must hold [{self.B}*{self.L}, d], weight [{self.V}, d]")
+        if not getattr(self, "_lm_reserved", False):
+            _check(_lib().eb_lmhead_reserve(self._h, d), "eb_lmhead_reserve")
+            self._lm_reserved = True
+        _check(_lib().eb_lmhead_step(
+            self._h, C.c_void_p(hidden.data_ptr()), C.c_void_p(weight.data_ptr()), d, int(step),
+            self._ptr(canvas, torch.int32, (self.B, self.L), "canvas"),
+            self._ptr(committed, torch.uint8, (self.B, self.L), "committed"),
+            self._ptr(entropies, torch.float32, (self.B, self.L), "entropies"),
+            self._ptr(argmax, torch.int32, (self.B, self.L), "argmax"),
+            self._ptr(stop_flags, torch.uint8, (self.B,), "stop_flags"), self._stream()),
+            "eb_lmhead_step")
 
     # -- vocabulary-sharded logits ---------------------------------------------
     def slice_records(self):

@@ -231,6 +231,12 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
   return p;
 }
 
+__device__ __forceinline__ uint64_t evict_last_policy() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+
 __device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes,
                                           uint64_t* bar, uint64_t policy) {
   asm volatile(

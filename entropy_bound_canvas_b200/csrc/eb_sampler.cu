@@ -19,7 +19,10 @@
 #include <mutex>
 #include <new>
 
+#include <cudaTypedefs.h>
+
 #include "eb_finish.cuh"
+#include "eb_lmhead.cuh"
 #include "eb_stream.cuh"
 
 namespace {
@@ -65,6 +68,10 @@ void device_setup(DeviceAttrs& d, int device) {
       cudaFuncSetAttribute(ebk::stream_kernel<ebk::kBF16>,
                            cudaFuncAttributeMaxDynamicSharedMemorySize, optin) != cudaSuccess ||
       cudaFuncSetAttribute(ebk::combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::lmhead_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           optin) != cudaSuccess ||
+      cudaFuncSetAttribute(ebk::lmhead_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            optin) != cudaSuccess) {
     cudaGetLastError();
     d.rc = EB_ERR_CUDA;
@@ -114,6 +121,9 @@ struct eb_sampler {
   float* pmax = nullptr;
   int last_step = -1;
   cudaEvent_t split_event = nullptr;  // recorded after the step's kernel when set
+  // the LM-head step's per-(position, vocabulary range) records
+  ebk::SliceRecord* lm_rec = nullptr;
+  int lm_split = 0;
 };
 
 namespace {
@@ -412,6 +422,76 @@ bool is_slice(const eb_sampler* h) {
   return h->cfg.vocab_offset != 0 || h->V_tot != h->cfg.V;
 }
 
+// ---------------------------------------------------------------------------
+// LM-head step: tensor maps and launch
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    cudaGetLastError();
+  });
+  return fn;
+}
+
+// A bf16 matrix [outer][inner] (inner contiguous), read in boxes of
+// box_outer x 64 with the 128-byte swizzle the MMA descriptors expect.
+bool make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+               uint32_t box_outer) {
+  PFN_cuTensorMapEncodeTiled_v12000 enc = tmap_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)ebk::kLmBK, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
+// Sizes the LM-head kernels accept: the hidden size a multiple of 64, the
+// vocabulary a multiple of 256 (one MMA N tile), 16-byte aligned operands.
+int lm_check(const void* hidden, const void* weight, int64_t rows, int64_t V, int64_t d) {
+  if (!hidden || !weight || rows < 1 || V < ebk::kLmBN || d < ebk::kLmBK)
+    return EB_ERR_INVALID_ARG;
+  if (d % ebk::kLmBK != 0 || V % ebk::kLmBN != 0) return EB_ERR_UNSUPPORTED;
+  if ((uintptr_t)hidden % 16 != 0 || (uintptr_t)weight % 16 != 0) return EB_ERR_INVALID_ARG;
+  if (rows > (1ll << 30) || V > (1ll << 30) || d > (1 << 20)) return EB_ERR_OVERFLOW;
+  return EB_OK;
+}
+
+// Vocabulary ranges per 128-row tile: one CTA per SM over all tiles.
+int lm_split_count(int sms, int64_t rows, int64_t V) {
+  const int n_mt = (int)((rows + ebk::kLmBM - 1) / ebk::kLmBM);
+  const int n_nt = (int)(V / ebk::kLmBN);
+  return std::max(1, std::min(n_nt, sms / std::max(1, n_mt)));
+}
+
+int lm_launch(bool sampler, const DeviceAttrs& d, const void* hidden, const void* weight,
+              ebk::LmArgs& p, cudaStream_t st) {
+  CUtensorMap th, tw;
+  if (!make_tmap(&th, hidden, (uint64_t)p.d, (uint64_t)p.rows, ebk::kLmBM) ||
+      !make_tmap(&tw, weight, (uint64_t)p.d, (uint64_t)p.V, ebk::kLmBN))
+    return EB_ERR_CUDA;
+  const size_t smem = ebk::lm_layout(sampler).total;
+  if (smem > d.optin) return EB_ERR_UNSUPPORTED;
+  const int n_mt = (p.rows + ebk::kLmBM - 1) / ebk::kLmBM;
+  void* args[] = {&th, &tw, &p};
+  const void* fn = sampler ? reinterpret_cast<const void*>(&ebk::lmhead_kernel<true>)
+                           : reinterpret_cast<const void*>(&ebk::lmhead_kernel<false>);
+  if (cudaLaunchKernel(fn, dim3(n_mt * p.n_split), dim3(ebk::kLmThreads), args, smem, st) !=
+      cudaSuccess)
+    return EB_ERR_CUDA;
+  return EB_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -503,6 +583,99 @@ int eb_sampler_combine(eb_sampler_t* h, const void* records, int n_slices, int s
 }
 
 size_t eb_slice_record_bytes(void) { return sizeof(ebk::SliceRecord); }
+
+int eb_lmhead_logits(const void* hidden, const void* weight, int32_t rows, int32_t V, int32_t d,
+                     float* logits, void* stream) {
+  int rc = lm_check(hidden, weight, rows, V, d);
+  if (rc != EB_OK) return rc;
+  if (!logits || (uintptr_t)logits % 16 != 0) return EB_ERR_INVALID_ARG;
+  int device = 0;
+  if (cudaGetDevice(&device) != cudaSuccess) return EB_ERR_CUDA;
+  DeviceAttrs* da = nullptr;
+  if ((rc = device_attrs(device, &da)) != EB_OK) return rc;
+  ebk::LmArgs p;
+  std::memset(&p, 0, sizeof(p));
+  p.a.wait_ns = ebk::kWaitLimitNs;
+  p.a.status = nullptr;
+  p.logits_out = logits;
+  p.rows = rows;
+  p.V = V;
+  p.d = d;
+  p.n_split = lm_split_count(da->sms, rows, V);
+  return lm_launch(false, *da, hidden, weight, p, (cudaStream_t)stream);
+}
+
+int eb_lmhead_reserve(eb_sampler_t* h, int32_t d) {
+  if (!h || d < ebk::kLmBK || d % ebk::kLmBK != 0) return EB_ERR_INVALID_ARG;
+  if (is_slice(h) || h->cfg.V % ebk::kLmBN != 0) return EB_ERR_UNSUPPORTED;
+  if (h->lm_rec) return EB_OK;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  const int64_t rows = (int64_t)h->cfg.B * h->cfg.L;
+  const int split = lm_split_count(h->sms, rows, h->cfg.V);
+  void* ptr = nullptr;
+  if (cudaMalloc(&ptr, (size_t)split * (size_t)rows * sizeof(ebk::SliceRecord)) != cudaSuccess) {
+    cudaGetLastError();
+    return EB_ERR_OUT_OF_MEMORY;
+  }
+  h->lm_rec = static_cast<ebk::SliceRecord*>(ptr);
+  h->lm_split = split;
+  return EB_OK;
+}
+
+int eb_lmhead_step(eb_sampler_t* h, const void* hidden, const void* weight, int32_t d, int step,
+                   int32_t* canvas, uint8_t* committed, float* entropies, int32_t* argmax,
+                   uint8_t* stop_flags, void* stream) {
+  if (!h || !canvas || !committed || !entropies || !argmax || !stop_flags)
+    return EB_ERR_INVALID_ARG;
+  const eb_config_t& c = h->cfg;
+  const int64_t rows = (int64_t)c.B * c.L;
+  int rc = lm_check(hidden, weight, rows, c.V, d);
+  if (rc != EB_OK) return rc;
+  if (!h->lm_rec) return EB_ERR_INVALID_ARG;  // eb_lmhead_reserve first
+  if (is_slice(h)) return EB_ERR_UNSUPPORTED;
+  if (step < 0 || step >= c.num_steps) return EB_ERR_INVALID_ARG;
+  if (step != 0 && step != h->last_step + 1) return EB_ERR_STEP_ORDER;
+  DeviceGuard guard(h->device);
+  if (!guard.ok) return EB_ERR_CUDA;
+  DeviceAttrs* da = nullptr;
+  if ((rc = device_attrs(h->device, &da)) != EB_OK) return rc;
+  cudaStream_t st = (cudaStream_t)stream;
+
+  // the fused contraction and sampler pass: one record per (position,
+  // vocabulary range)
+  ebk::LmArgs p;
+  std::memset(&p, 0, sizeof(p));
+  fill_args(h, p.a, step);
+  p.a.committed = committed;
+  p.a.stop_flags = stop_flags;
+  p.rec = h->lm_rec;
+  p.rows = (int)rows;
+  p.V = c.V;
+  p.d = d;
+  p.n_split = h->lm_split;
+  if ((rc = lm_launch(true, *da, hidden, weight, p, st)) != EB_OK) return rc;
+  // the active canvases, then the records merged in vocabulary order and the
+  // canvas decisions
+  StepArgs a;
+  fill_args(h, a, step);
+  a.canvas = canvas;
+  a.committed = committed;
+  a.H_out = entropies;
+  a.amax_out = argmax;
+  a.stop_flags = stop_flags;
+  ebk::active_index_kernel<<<1, 256, 0, st>>>(stop_flags, c.B, h->act_index);
+  if (cudaGetLastError() != cudaSuccess) return EB_ERR_CUDA;
+  const int32_t* act_index = h->act_index;
+  const ebk::SliceRecord* rec = h->lm_rec;
+  int n_slices = h->lm_split;
+  void* cargs[] = {&a, &act_index, &rec, &n_slices};
+  if (cudaLaunchKernel(h->combine.fn, dim3(h->combine.grid), dim3(ebk::kEpiThreads), cargs,
+                       h->combine.smem, st) != cudaSuccess)
+    return EB_ERR_CUDA;
+  h->last_step = step;
+  return EB_OK;
+}
 
 int eb_canvas_done(eb_sampler_t* h, const uint8_t* stop_flags, int b, int* done, void* stream) {
   if (!h || !stop_flags || !done) return EB_ERR_INVALID_ARG;
@@ -608,6 +781,7 @@ void eb_sampler_destroy(eb_sampler_t* h) {
   {
     DeviceGuard guard(h->device);
     if (h->ws) cudaFree(h->ws);
+    if (h->lm_rec) cudaFree(h->lm_rec);
   }
   delete h;
 }

@@ -263,6 +263,46 @@ int eb_sampler_combine(eb_sampler_t* h, const void* records, int n_slices, int s
                        uint8_t* stop_flags, void* stream);
 size_t eb_slice_record_bytes(void);
 
+/* The sampler fused into the decoder's LM head: a step from the last hidden
+   states instead of from logits.  The logits z = h W^T are formed on the
+   tensor cores (tcgen05, bf16 in, fp32 accumulate) tile by tile and reduced
+   on chip -- maximum, argmax, the entropy sums, the two-level Gumbel draw --
+   so they never reach HBM; then the canvas decisions run as in
+   eb_sampler_step (diffusers "DiffusionGemma" page, `__call__` parameters:
+   the pipeline's logits are the decoder's [batch, canvas_length,
+   vocab_size] output; model card, summary table: vocabulary about 262K).
+     hidden  [B*L][d] bf16, device memory, 16-byte aligned, row-major (row =
+             canvas b, position l in the handle's order), read only;
+     weight  [V][d] bf16, device memory, 16-byte aligned, row-major (the LM
+             head, one row per vocabulary id), read only;
+     d       hidden size, a multiple of 64; V (the handle's) a multiple of
+             256; the handle must cover the whole vocabulary (no slice);
+     canvas .. stop_flags, stream: as in eb_sampler_step.
+   The results equal eb_sampler_step on the logits z computed in fp32: the
+   argmax and the draw exactly wherever z is (for example when every partial
+   sum of h W^T is exactly representable), the entropies to rounding.
+   eb_lmhead_reserve(h, d) allocates the handle's per-(position, vocabulary
+   range) records once, before the first eb_lmhead_step (EB_ERR_INVALID_ARG
+   otherwise); eb_lmhead_step itself allocates nothing and never
+   synchronises.  Step order as in eb_sampler_step.  Errors:
+   EB_ERR_UNSUPPORTED for d or V not multiples of 64 / 256 or a slice
+   handle, EB_ERR_INVALID_ARG for NULL or misaligned pointers, bad steps.
+   A pipeline wait that runs out sets EB_STATUS_TIMEOUT as in the stream
+   kernel.  No counterpart in the pages' pipeline, which forms the logits
+   first; this is the same step with the logits kept on chip. */
+int eb_lmhead_reserve(eb_sampler_t* h, int32_t d);
+int eb_lmhead_step(eb_sampler_t* h, const void* hidden, const void* weight, int32_t d, int step,
+                   int32_t* canvas, uint8_t* committed, float* entropies, int32_t* argmax,
+                   uint8_t* stop_flags, void* stream);
+
+/* Diagnostic form of the LM-head kernel's contraction: logits [rows][V]
+   fp32 (device memory, 16-byte aligned, caller-owned) = hidden [rows][d] x
+   weight[V][d]^T, both bf16 as in eb_lmhead_step, on the current device and
+   `stream`.  Same size rules; no handle.  It lets a caller (and the tests)
+   check the tensor-core contraction apart from the sampler. */
+int eb_lmhead_logits(const void* hidden, const void* weight, int32_t rows, int32_t V, int32_t d,
+                     float* logits, void* stream);
+
 /* Profiling hook.  When `event` (a cudaEvent_t passed as void*, owned by
    the caller) is non-NULL, every following eb_sampler_step records it on
    its stream right after the step's kernel, so that the caller can time that

@@ -250,6 +250,24 @@ def sample_flat(cfg: Config, row, inv_T: float, b: int, l: int, s: int):
 
 # --------------------------------------------------------------------------- canvas state
 
+def lmhead_logits(hidden_bits, weight_bits):
+    """The decoder's logits from its last hidden states and the LM head:
+    z[row, v] = sum_k h[row, k] W[v, k], in float64 (diffusers "DiffusionGemma"
+    page, `__call__` parameters: the pipeline's logits are the decoder's
+    [batch, canvas_length, vocab_size] output; model card, summary table:
+    a vocabulary of about 262K).  Inputs are bf16 bit patterns (uint16
+    [rows, d] and [V, d]); the product is numpy's float64 matrix product,
+    which is exact for inputs whose products and sums are exactly
+    representable (the synthetic recipe's multiples of 1/64)."""
+    return decode_bf16(hidden_bits) @ decode_bf16(weight_bits).T
+
+
+def decode_bf16(bits):
+    """bf16 bit patterns (uint16) -> float64 values (exact)."""
+    u = np.ascontiguousarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return u.view(np.float32).astype(np.float64)
+
+
 class State:
     """Per-canvas sampler state the oracle carries between steps."""
 
