@@ -22,7 +22,9 @@ runs its own canvas (global canvas index = rank): no data-path collective,
 weak scaling.
 
 At N = 1 the other large workloads (serve 8x, br 4x, stress 32x fp32) are
-timed afterwards as whole 48-step trajectories and reported under "configs".
+timed afterwards as whole 48-step trajectories and reported under "configs",
+with the sampler fused into the LM head (hidden size 2560, 1 and 8 canvases:
+"lmhead", "lmhead8") and its unfused counterpart.
 
 --impl reference times the CPU oracle (the float64 restatement in oracle/)
 on the host cores, rank 0 only, on bounded samples of the same workload.
@@ -46,6 +48,7 @@ METRIC = "canvas positions sampled/sec and HBM GB/s (% of B200 peak), 256x262144
 UNIT = "positions/s"
 WORKLOAD = "canvas"
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 
 
 def parse():
@@ -61,12 +64,15 @@ def parse():
                    help="timed regions of exactly K steps (median reported); 0 = automatic")
     p.add_argument("--configs", default="all",
                    help="other workloads timed after the headline one: all, none, or a list "
-                        "of serve,br,stress (N = 1 only by default)")
+                        "of serve,br,stress,lmhead,lmhead8 (N = 1 only by default)")
     p.add_argument("--split-v", action="store_true",
                    help="vocabulary-sharded canvas: each rank holds a slice of the vocabulary; "
                         "a step is the slice pass, one all-gather of the records, the combine")
     p.add_argument("--profile", action="store_true",
                    help="small case for ncu: logits of steps 0-2 only, three eager steps")
+    p.add_argument("--profile-lmhead", action="store_true",
+                   help="small case for ncu: three LM-head steps, 1 x 256 positions, "
+                        "V = 32768, hidden size 2560")
     return p.parse_args()
 
 
@@ -78,6 +84,85 @@ def peaks():
         return float(d["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 tensor peak (TFLOP/s): the measured burst figure, else the
+    pool's fallback."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, "fallback"
+
+
+def run_lmhead_config(E, synth, dev, B, d, barrier, max_over_ranks):
+    """The sampler fused into the LM head (eb_lmhead_step): 48-step
+    trajectories from the hidden states of the synthetic recipe (hidden size
+    d, an assumption: the pages give none), replayed from a CUDA graph; and,
+    for context, the same steps unfused (cuBLAS bf16 GEMM to bf16 logits,
+    then the sampler step)."""
+    import torch
+
+    from synth import lmhead as LM
+    w = synth.WORKLOADS["canvas"].replace(B=B, seed=31)
+    N = w.num_steps
+    wc = LM.weight_codes(w.V, d, seed=w.seed)
+    W = LM.to_bf16(wc).to(dev)
+    hs = [LM.to_bf16(LM.hidden_codes(wc, w.B, w.L, s, N, seed=w.seed)).to(dev) for s in range(N)]
+    del wc
+    eb = E.EBSampler(w.B, w.L, w.V, device=dev, **w.sampler_config())
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    lg = torch.empty((w.B, w.L, w.V), dtype=torch.bfloat16, device=dev)
+
+    def fused():
+        eb.init_canvas(canvas, committed, stop)
+        for s in range(N):
+            eb.lmhead_step(hs[s], W, s, canvas, committed, H, amax, stop)
+
+    def unfused():
+        eb.init_canvas(canvas, committed, stop)
+        for s in range(N):
+            torch.matmul(hs[s], W.T, out=lg.view(w.B * w.L, w.V))
+            eb.step(lg, s, canvas, committed, H, amax, stop)
+
+    out = {}
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(side):
+            fn()
+            torch.cuda.synchronize()
+            with torch.cuda.graph(g, stream=side):
+                fn()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        times = timed_regions(g.replay, 5, barrier, torch.cuda.current_stream(dev))
+        out[name] = max_over_ranks(statistics.median(times)) / N
+        del g
+    status = eb.status()
+    eb.close()
+    flop = 2.0 * w.B * w.L * w.V * d
+    peak, kind = tensor_peak()
+    tfl = flop / (out["fused"] * 1e-3) / 1e12
+    return {
+        "workload": f"{B} x 256 x 262144, hidden size {d} (bf16 hidden states and LM head), "
+                    "logits formed and reduced on chip",
+        "value": w.B * w.L / (out["fused"] * 1e-3), "unit": UNIT,
+        "ms_per_step": out["fused"], "steps": N, "status": status,
+        "unfused_ms_per_step": out["unfused"],
+        "roofline": {"bound": "tensor", "achieved": tfl, "peak": peak, "unit": "TFLOP/s",
+                     "frac": tfl / peak, "kernel": "ebk::lmhead_kernel<true>",
+                     "flop_per_step": flop,
+                     "peak_source": f"{kind} MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)"},
+    }
 
 
 def kernel_source_hash():
@@ -355,6 +440,8 @@ def roofline_of(kernel, launches, bytes_total, region_ms, peak, peak_kind):
             "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"}
 
 
+LMHEAD_D = 2560  # hidden size of the LM-head configs (the pages give none)
+
 EXTRA = {
     # name -> (rotate buffers or None, description)
     "serve": (None, "8 x 256 x 262144 bf16 per GPU, staggered stops, 48 steps resident"),
@@ -524,10 +611,16 @@ def run_ours(args):
     # the other large workloads: full 48-step trajectories from one graph each
     extra = {}
     names = [] if args.configs == "none" else (
-        list(EXTRA) if args.configs == "all" else args.configs.split(","))
+        list(EXTRA) + ["lmhead", "lmhead8"] if args.configs == "all"
+        else args.configs.split(","))
     if world > 1 and args.configs == "all":
         names = []  # the scaling runs time the headline workload only
     for name in names:
+        if name.startswith("lmhead"):
+            Bx = 8 if name == "lmhead8" else 1
+            extra[name] = run_lmhead_config(E, synth, dev, Bx, LMHEAD_D, barrier, max_over_ranks)
+            torch.cuda.empty_cache()
+            continue
         rotate, desc = EXTRA[name]
         wx = synth.WORKLOADS[name]
         tx = Trajectory(E, synth, wx, dev, rank, rotate=rotate)
@@ -695,10 +788,38 @@ def run_profile_case():
     print("profile case done")
 
 
+def run_profile_lmhead_case():
+    """Three LM-head steps of a small case (1 x 256 positions, V = 32768,
+    d = 2560; about 0.2 GB on the device)."""
+    import torch
+
+    import entropy_bound_canvas_b200 as E
+    import synth
+    from synth import lmhead as LM
+    dev = torch.device("cuda", 0)
+    w = synth.WORKLOADS["canvas"].replace(V=32768, seed=31)
+    wc = LM.weight_codes(w.V, LMHEAD_D, seed=w.seed)
+    W = LM.to_bf16(wc).to(dev)
+    eb = E.EBSampler(w.B, w.L, w.V, device=dev, **w.sampler_config())
+    canvas, committed, stop = eb.new_canvas()
+    H, amax = eb.outputs()
+    eb.init_canvas(canvas, committed, stop)
+    for s in range(3):
+        h = LM.to_bf16(LM.hidden_codes(wc, w.B, w.L, s, w.num_steps, seed=w.seed)).to(dev)
+        eb.lmhead_step(h, W, s, canvas, committed, H, amax, stop)
+    torch.cuda.synchronize()
+    assert eb.status() == 0
+    eb.close()
+    print("lmhead profile case done")
+
+
 def main():
     args = parse()
     if args.profile:
         run_profile_case()
+        return
+    if args.profile_lmhead:
+        run_profile_lmhead_case()
         return
     if args.impl == "reference":
         run_reference(args)
