@@ -359,7 +359,9 @@ __global__ void __launch_bounds__(kLmThreads, 1)
     const float c2 = a.c2;
     for (int t = 0; t < n_tiles; ++t) {
       const int buf = t & 1;
-      if (!mbar_wait(&acc_full[buf], (uint32_t)(t / 2) & 1u, a.wait_ns, abort_flag)) {
+      // a warp-uniform outcome: the TMEM loads below need the whole warp
+      if (!__all_sync(0xffffffffu,
+                      mbar_wait(&acc_full[buf], (uint32_t)(t / 2) & 1u, a.wait_ns, abort_flag))) {
         if (lane == 0) fail();
         break;
       }
@@ -375,6 +377,7 @@ __global__ void __launch_bounds__(kLmThreads, 1)
         float z[64];
         {
           float lo[32], hi[32];
+          __syncwarp();  // tcgen05.ld is warp-wide: every lane, converged
           tc_ld32(taddr + (uint32_t)(g * kGroup), lo);
           tc_ld32(taddr + (uint32_t)(g * kGroup + 32), hi);
           tc_wait_ld();
@@ -392,65 +395,67 @@ __global__ void __launch_bounds__(kLmThreads, 1)
           for (int i = 0; i < 16; ++i) out[i] = make_float4(z[4 * i], z[4 * i + 1], z[4 * i + 2], z[4 * i + 3]);
           continue;
         }
-        // group maximum and its lowest index
-        float m8[8];
+        if constexpr (SAMPLER) {
+          // group maximum and its lowest index
+          float m8[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          float m = z[8 * j];
+          for (int j = 0; j < 8; ++j) {
+            float m = z[8 * j];
 #pragma unroll
-          for (int i = 1; i < 8; ++i) m = fmaxf(m, z[8 * j + i]);
-          m8[j] = m;
-        }
-        const float mg = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                               fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-        uint32_t eq_lo = 0u, eq_hi = 0u;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          eq_lo |= (z[i] == mg ? 1u : 0u) << i;
-          eq_hi |= (z[32 + i] == mg ? 1u : 0u) << i;
-        }
-        const int ig = eq_lo ? __ffs(eq_lo) - 1 : 31 + __ffs(eq_hi);
-        if (mg > st.M) {  // a new maximum: rescale the state to it
-          if (st.M > -INFINITY) {
-            const float dd = (st.M - mg) * c2;
-            const float f = ex2(dd);
-            st.W = f * fmaf(dd, st.S, st.W);
-            st.S *= f;
-            st.R *= f;
+            for (int i = 1; i < 8; ++i) m = fmaxf(m, z[8 * j + i]);
+            m8[j] = m;
           }
-          st.M = mg;
-          st.amax = v0 + ig;
-        }
-        // the group's sums relative to the maximum (z - M exact for the
-        // largest terms, so the maximum's own term is exactly 1)
-        float s8[8], w8[8];
+          const float mg = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                 fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          uint32_t eq_lo = 0u, eq_hi = 0u;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) s8[j] = w8[j] = 0.f;
+          for (int i = 0; i < 32; ++i) {
+            eq_lo |= (z[i] == mg ? 1u : 0u) << i;
+            eq_hi |= (z[32 + i] == mg ? 1u : 0u) << i;
+          }
+          const int ig = eq_lo ? __ffs(eq_lo) - 1 : 31 + __ffs(eq_hi);
+          if (mg > st.M) {  // a new maximum: rescale the state to it
+            if (st.M > -INFINITY) {
+              const float dd = (st.M - mg) * c2;
+              const float f = ex2(dd);
+              st.W = f * fmaf(dd, st.S, st.W);
+              st.S *= f;
+              st.R *= f;
+            }
+            st.M = mg;
+            st.amax = v0 + ig;
+          }
+          // the group's sums relative to the maximum (z - M exact for the
+          // largest terms, so the maximum's own term is exactly 1)
+          float s8[8], w8[8];
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float d = (z[i] - st.M) * c2;
-          const float e = ex2(d);
-          s8[i & 7] += e;
-          w8[i & 7] = fmaf(e, d, w8[i & 7]);
-        }
-        const float Sg = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
-        const float Wg = ((w8[0] + w8[1]) + (w8[2] + w8[3])) + ((w8[4] + w8[5]) + (w8[6] + w8[7]));
-        st.S += Sg;
-        st.W += Wg;
-        if (samp) {  // the group-level race (strict: the earlier group keeps a tie)
-          const uint32_t x = pick_word(gw, (uint32_t)g);
-          if (!(Sg * 1.0001f <= st.R * one_minus_u(x))) {
-            const float E = -logf(uniform_open(x));
-            if (Sg > st.R * E) {
-              st.R = __fdividef(Sg, E);
-              st.gb = v0 / kGroup;
+          for (int j = 0; j < 8; ++j) s8[j] = w8[j] = 0.f;
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                reinterpret_cast<float2*>(zrow)[i] = make_float2(z[2 * i], z[2 * i + 1]);
+          for (int i = 0; i < 64; ++i) {
+            const float d = (z[i] - st.M) * c2;
+            const float e = ex2(d);
+            s8[i & 7] += e;
+            w8[i & 7] = fmaf(e, d, w8[i & 7]);
+          }
+          const float Sg = ((s8[0] + s8[1]) + (s8[2] + s8[3])) + ((s8[4] + s8[5]) + (s8[6] + s8[7]));
+          const float Wg = ((w8[0] + w8[1]) + (w8[2] + w8[3])) + ((w8[4] + w8[5]) + (w8[6] + w8[7]));
+          st.S += Sg;
+          st.W += Wg;
+          if (samp) {  // the group-level race (strict: the earlier group keeps a tie)
+            const uint32_t x = pick_word(gw, (uint32_t)g);
+            if (!(Sg * 1.0001f <= st.R * one_minus_u(x))) {
+              const float E = -logf(uniform_open(x));
+              if (Sg > st.R * E) {
+                st.R = __fdividef(Sg, E);
+                st.gb = v0 / kGroup;
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                  reinterpret_cast<float2*>(zrow)[i] = make_float2(z[2 * i], z[2 * i + 1]);
+              }
             }
           }
-        }
-      }
+              }
+}
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[buf]);

@@ -563,6 +563,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   // on the stream may be scheduled from now on, wherever an SM has room: it
   // waits for this grid's completion in turn before reading anything this
   // grid writes.
+  const int G = gridDim.x;
   griddep_wait();
   griddep_launch_dependents();
   // Every warp counts the active canvases itself (no block barrier); the
@@ -577,7 +578,6 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     if (atomicAdd(&ctrl->nread, 1) == Sh::kThreads / 32 - 1 && a.run_epilogue)
       atomicAdd(a.sync_cnt, 1);
   }
-  const int G = gridDim.x;
   const unsigned long long NG =
       (unsigned long long)n_act * (unsigned long long)a.L * (unsigned long long)a.ng;
   const unsigned long long g_lo = range_start(blockIdx.x, NG, G);
@@ -596,9 +596,11 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
 
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
   const char* logits = reinterpret_cast<const char*>(a.logits);
-  const long long r_first = (long long)(g_lo / (unsigned long long)a.ng);
-  const long long r_end =
-      g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
+  // the range's first row and one past its last (roles that need them)
+  auto row_range = [&](long long& r_first, long long& r_end) {
+    r_first = (long long)(g_lo / (unsigned long long)a.ng);
+    r_end = g_hi > g_lo ? (long long)((g_hi - 1ull) / (unsigned long long)a.ng) + 1 : r_first;
+  };
   auto row_of = [&](long long r, int& bi, int& l) {
     const int ai = (int)(r / a.L);
     l = (int)(r - (long long)ai * a.L);
@@ -684,6 +686,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // stage's header and makes the stage's second arrival.  The committed
     // flags of the range's first 32 rows are loaded at once, at the start.
     const int n_tiles = wait_ready() ? ctrl->n_sub / Sh::kSubPerStage : 0;
+    long long r_first, r_end;
+    row_range(r_first, r_end);
     uint32_t open_bits = 0;
     if (!a.greedy) {
       const long long r = r_first + lane;
@@ -699,7 +703,9 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     long long row_seen = -1;
     int samp = 0;
     for (int k = 0; k < n_tiles; ++k, words_done = k) {
-      if (!wait_counter_above(&ctrl->issued, k, a.wait_ns)) {
+      // every lane waits (bounded); the warp acts on the vote, so that a
+      // limit running out for some lanes only still ends the loop for all
+      if (!__all_sync(0xffffffffu, wait_counter_above(&ctrl->issued, k, a.wait_ns))) {
         if (lane == 0) {
           atomicOr(a.status, kStatusTimeout);
           *(volatile int*)&ctrl->abort = 1;
@@ -742,6 +748,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     // Finisher f takes the rows q = f, f + kFinishers, ... of the range, so
     // that rows completed close together (at the end of the range) are
     // finished in parallel.
+    long long r_first, r_end;
+    row_range(r_first, r_end);
     const int nrows = wait_ready() ? (int)(r_end - r_first) : 0;
     const int f = warp - (NW + 2);
     for (int q = f; q < nrows; q += Sh::kFinishers) {
@@ -840,6 +848,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   } else {
     // ------------------------------------------------------------ consumers
     const int n_sub = wait_ready() ? ctrl->n_sub : 0;
+    long long r_first, r_end;
+    row_range(r_first, r_end);
     long long cur_r = -1;
     long long next_r = r_first;  // first row of the range this warp still owes a deposit
     int sampling = 0;
@@ -907,9 +917,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       const int k = u / Sh::kSubPerStage;
       const int sub = u & (Sh::kSubPerStage - 1);
       const int st = k % kStages;
-      if (!mbar_wait(&full[st], (uint32_t)(k / kStages) & 1u, a.wait_ns, &ctrl->abort)) {
-        fail = true;
-        break;
+      // one try in every lane, agreed by a vote; when it is not yet
+      // complete, a bounded wait in every lane and a second vote
+      {
+        const uint32_t par = (uint32_t)(k / kStages) & 1u;
+        if (!__all_sync(0xffffffffu, mbar_try_wait(&full[st], par)) &&
+            !__all_sync(0xffffffffu, mbar_wait(&full[st], par, a.wait_ns, &ctrl->abort))) {
+          fail = true;
+          break;
+        }
       }
       const TileMeta m = meta[st];
       const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
@@ -1023,7 +1039,9 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
-    if (!fail && !*(volatile int*)&ctrl->abort) {
+    // The abort flag may change while the lanes read it: the warp acts on
+    // one vote (the deposits below are warp-wide).
+    if (__all_sync(0xffffffffu, !fail && !*(volatile int*)&ctrl->abort)) {
       if (cur_r >= 0) {
         if (!deposit(cur_r, false)) fail = true;
         next_r = cur_r + 1;
