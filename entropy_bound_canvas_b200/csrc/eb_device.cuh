@@ -136,23 +136,67 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// One test of the phase that may suspend the thread for up to hint_ns; the
+// thread resumes as soon as the phase completes.
+__device__ __forceinline__ bool mbar_try_wait_for(uint64_t* bar, uint32_t parity,
+                                                  uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Every wait gives up after a limit and reports a timeout: the pipeline
 // waits after the step's configured limit (2 s unless a test shortens it),
 // the drain of copies still in flight at a kernel's exit after kDrainLimitNs.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 constexpr uint64_t kDrainLimitNs = 2000000000ull;
+// Suspension asked of one test (the limit and the abort flag are looked at
+// between tests).
+constexpr uint32_t kSuspendHintNs = 20000;
 
-// Gives up (false) after limit_ns, or once *abort is set when abort is given
-// (checked only on the slow path).
+// One test of the phase that never suspends the thread.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Gives up (false) after limit_ns, or once *abort is set when abort is given.
+// A suspended test may last until the phase completes (whatever its hint):
+// the limit bounds a wait for a phase that does not complete.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
                                           uint64_t limit_ns = kWaitLimitNs,
                                           const int* abort = nullptr) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait_for(bar, parity, kSuspendHintNs)) return true;
   const uint64_t t0 = global_ns();
   for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i)
-      if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_for(bar, parity, kSuspendHintNs)) return true;
+    if (abort != nullptr && *(const volatile int*)abort) return false;
+    if (global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+// mbar_wait, except that a limit shorter than kSuspendHintNs is kept with
+// tests that never suspend and the clock read after each: such a limit runs
+// out whenever the phase is not complete at the first test.
+__device__ __noinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                             const int* abort) {
+  if (limit_ns >= kSuspendHintNs) return mbar_wait(bar, parity, limit_ns, abort);
+  const uint64_t t0 = global_ns();
+  for (;;) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (abort != nullptr && *(const volatile int*)abort) return false;
     if (global_ns() - t0 > limit_ns) return false;
   }
@@ -184,43 +228,6 @@ __device__ __forceinline__ int atom_add_acq_rel_gpu(int* p, int v) {
   int old;
   asm volatile("atom.acq_rel.gpu.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(p), "r"(v) : "memory");
   return old;
-}
-
-// Waits (bounded like mbar_wait) until *p > k.
-__device__ __forceinline__ bool wait_counter_above(const int* p, int k,
-                                                   uint64_t limit_ns = kWaitLimitNs) {
-  if (ld_acquire_shared(p) > k) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-      __nanosleep(32);
-      if (ld_acquire_shared(p) > k) return true;
-    }
-    if (global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-// Waits (bounded) until *p == v.
-__device__ __forceinline__ bool wait_counter_equal(const int* p, int v,
-                                                   uint64_t limit_ns = kWaitLimitNs) {
-  if (ld_acquire_shared(p) == v) return true;
-  const uint64_t t0 = global_ns();
-  for (;;) {
-#pragma unroll 1
-    for (int i = 0; i < 32; ++i) {
-      __nanosleep(20);
-      if (ld_acquire_shared(p) == v) return true;
-    }
-    if (global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-// Shared-memory add with release semantics (publishes this thread's earlier
-// shared-memory writes to a thread that reads the counter with acquire).
-__device__ __forceinline__ void red_release_shared_add(int* p, int v) {
-  asm volatile("red.release.cta.shared::cta.add.s32 [%0], %1;" ::"r"(smem_u32(p)), "r"(v)
-               : "memory");
 }
 
 // L2 policy for data read exactly once: evict it first, so that a stream

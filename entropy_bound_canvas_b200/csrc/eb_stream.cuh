@@ -83,7 +83,6 @@ struct StreamCtrl {
   int words_arrived;  // tiles whose second (header) arrival was made
   int n_epi;          // canvases whose decisions this CTA runs
   int epi_ok;         // every CTA of the grid has read the stop flags
-  int ready;          // the producer has published act, n_sub
   int nread;          // warps that have read the stop flags
 };
 
@@ -101,9 +100,9 @@ struct TileMeta {
 
 // A row slot: the consumer warps' deposits for one row of the CTA's range.
 struct RowSlot {
-  int q;      // CTA-relative row the slot accepts deposits for
-  int count;  // deposits made
-  int pad0, pad1;
+  int q;  // CTA-relative row the slot accepts deposits for
+  int pad0;
+  uint64_t full;  // one arrival per consumer warp's deposit
   Acc rec[EB_STREAM_CONSUMER_WARPS];
 };
 
@@ -119,7 +118,7 @@ __host__ __device__ inline StreamLayout stream_layout(int B) {
   StreamLayout y;
   uint32_t o = 0;
   y.bars = o;
-  o = align_up(o + 16u * kStages, 16);
+  o = align_up(o + 24u * kStages + 8u, 16);  // full, empty, described; ready
   y.ctrl = o;
   o = align_up(o + (uint32_t)sizeof(StreamCtrl), 16);
   y.meta = o;
@@ -528,6 +527,8 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   const StreamLayout lay = stream_layout<DT>(a.B);
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + lay.bars);
   uint64_t* empty = full + kStages;
+  uint64_t* described = empty + kStages;  // a tile's copy issued, its description written
+  uint64_t* ready = described + kStages;  // the active list and sub-tile count published
   StreamCtrl* ctrl = reinterpret_cast<StreamCtrl*>(smem + lay.ctrl);
   TileMeta* meta = reinterpret_cast<TileMeta*>(smem + lay.meta);
   uint32_t* words = reinterpret_cast<uint32_t*>(smem + lay.words);
@@ -541,17 +542,18 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     for (int st = 0; st < kStages; ++st) {
       mbar_init(&full[st], 2);  // the copy's arrival (+ bytes) and the header's
       mbar_init(&empty[st], Sh::kSubPerStage);
+      mbar_init(&described[st], 1);
     }
+    mbar_init(ready, 1);
     ctrl->abort = 0;
     ctrl->issued = 0;
     ctrl->words_arrived = 0;
     ctrl->n_epi = 0;
     ctrl->epi_ok = 0;
-    ctrl->ready = 0;
     ctrl->nread = 0;
     for (int i = 0; i < kSlots; ++i) {
       slots[i].q = i;
-      slots[i].count = 0;
+      mbar_init(&slots[i].full, NW);
     }
     fence_mbar_init();
   }
@@ -585,13 +587,12 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
   // The other roles start once the producer has published the active list
   // and the range's sub-tile count (right after its first copy).
   auto wait_ready = [&]() -> bool {
-    int ok = 1;
-    if (lane == 0 && !wait_counter_above(&ctrl->ready, 0, a.wait_ns)) {
+    const bool ok = __all_sync(0xffffffffu, mbar_wait_timed(ready, 0, a.wait_ns, &ctrl->abort));
+    if (!ok && lane == 0) {
       atomicOr(a.status, kStatusTimeout);
       *(volatile int*)&ctrl->abort = 1;
-      ok = 0;
     }
-    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+    return ok;
   };
 
   const size_t row_bytes = (size_t)a.V * (size_t)elt_bytes(DT);
@@ -618,7 +619,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       bool published = false;
       auto publish = [&]() {
         ctrl->n_sub = count_tiles(g_lo, g_hi, a.ng, Sh::kStageGroups) * Sh::kSubPerStage;
-        st_release_shared(&ctrl->ready, 1);
+        mbar_arrive(ready);
         published = true;
       };
       // Logits are read once: L2 evict-first, so that the stream does not push
@@ -665,6 +666,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         m.whole = a.vec_ok && (t.j0 + t.cnt) * kGroup <= a.V;
         meta[st] = m;
         st_release_shared(&ctrl->issued, k + 1);
+        mbar_arrive(&described[st]);
         if (!published) publish();
         ++k;
         if (++st == kStages) {
@@ -703,9 +705,13 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     long long row_seen = -1;
     int samp = 0;
     for (int k = 0; k < n_tiles; ++k, words_done = k) {
-      // every lane waits (bounded); the warp acts on the vote, so that a
-      // limit running out for some lanes only still ends the loop for all
-      if (!__all_sync(0xffffffffu, wait_counter_above(&ctrl->issued, k, a.wait_ns))) {
+      // every lane waits (bounded, suspended in the barrier rather than
+      // polling); the warp acts on the vote, so that a limit running out for
+      // some lanes only still ends the loop for all.  The phase is this
+      // warp's own next one: it waited for the stage's previous tile itself,
+      // and the stage's next tile needs this tile's header first.
+      if (!__all_sync(0xffffffffu, mbar_wait(&described[st], (uint32_t)(k / kStages) & 1u, a.wait_ns,
+                                             &ctrl->abort))) {
         if (lane == 0) {
           atomicOr(a.status, kStatusTimeout);
           *(volatile int*)&ctrl->abort = 1;
@@ -752,6 +758,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
     row_range(r_first, r_end);
     const int nrows = wait_ready() ? (int)(r_end - r_first) : 0;
     const int f = warp - (NW + 2);
+    static_assert(kSlots % Sh::kFinishers == 0, "a slot's rows must all go to one finisher");
     for (int q = f; q < nrows; q += Sh::kFinishers) {
       RowSlot* sl = &slots[q % kSlots];
       const long long r = r_first + q;
@@ -766,18 +773,10 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       // counter's round trip.)
       int pre = 0;
       if (sp.nseg > 1 && lane == 0) pre = ld_acquire_gpu(a.row_cnt + grow);
-      // the twelve deposits of row q
-      bool ok = true;
-      {
-        const uint64_t t0 = global_ns();
-        while (ld_acquire_shared(&sl->count) < NW) {
-          if (*(volatile int*)&ctrl->abort || global_ns() - t0 > a.wait_ns) {
-            ok = false;
-            break;
-          }
-          __nanosleep(32);
-        }
-      }
+      // the twelve deposits of row q: use q / kSlots of the slot, whose
+      // previous use this finisher waited for itself (a slot's rows all go
+      // to one finisher), and whose next needs this row's release first
+      const bool ok = mbar_wait(&sl->full, (uint32_t)(q / kSlots) & 1u, a.wait_ns, &ctrl->abort);
       if (!__all_sync(0xffffffffu, ok)) {
         if (lane == 0) {
           atomicOr(a.status, kStatusTimeout);
@@ -793,10 +792,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
       }
       warp_merge_acc(mine, a.c2);  // every lane ends with the CTA's merged state
       __syncwarp();
-      if (lane == 0) {
-        sl->count = 0;
-        st_release_shared(&sl->q, q + kSlots);
-      }
+      if (lane == 0) st_release_shared(&sl->q, q + kSlots);
       const char* rowp = logits + grow * row_bytes;
       // this part's candidate groups: loads in flight first
       const PartLoads pl = part_loads<DT>(a, mine, rowp, open && !a.greedy);
@@ -881,7 +877,7 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           } else {
             sl->rec[warp] = w;
           }
-          red_release_shared_add(&sl->count, 1);
+          mbar_arrive(&sl->full);
         }
       }
       return __shfl_sync(0xffffffffu, ok, 0) != 0;
@@ -927,10 +923,75 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           break;
         }
       }
-      const TileMeta m = meta[st];
       const int gl0 = sub * Sh::kSubGroups + lane, gl1 = gl0 + 32;
-      const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
       const uint32_t* wd = words + st * Sh::kStageGroups;
+      if (DT == kBF16 && a.vec_ok) {
+        // Rows on 16-byte boundaries: every tile's copy starts at the stage's
+        // first byte, so the lane's two groups and their race words are
+        // loaded together with the tile's description (one shared-memory
+        // round trip after the wait).  Both groups lie inside the stage
+        // whatever the tile's count; a group past the count is ignored.
+        const unsigned char* sb = ring + (size_t)st * Sh::kStageStride;
+        uint32_t G0[32], G1[32];
+        load_group_bf16(sb + (size_t)gl0 * 128, rot, G0);
+        load_group_bf16(sb + (size_t)gl1 * 128, rot, G1);
+        const uint32_t x0 = wd[gl0], x1 = wd[gl1];
+        const TileMeta m = meta[st];
+        if (m.whole) {
+          // the stage goes back to the producer; the row change (which may
+          // wait for a row slot) comes after the release
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&empty[st]);
+          if (!enter_row(m)) {
+            fail = true;
+            break;
+          }
+          const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;  // has1 implies has0
+          if (!has0) continue;
+          const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
+          // Both groups against one reference, the larger of the lane's
+          // maximum and theirs: a group raising it becomes the top group (the
+          // first on equal maxima), the other joins the rest; then the race,
+          // group 0 first.
+          const float mg0 = group_max_bf16(G0);
+          const float mg1 = has1 ? group_max_bf16(G1) : -INFINITY;
+          const bool v0 = mg0 > -INFINITY, v1 = mg1 > -INFINITY;  // not every logit -inf
+          if (!(v0 || v1)) continue;
+          const float mg = fmaxf(mg0, mg1);
+          const bool new_top = mg > A.M;
+          const float ref = new_top ? mg : A.M;
+          float S0, W0, S1, W1;
+          group_sums2_bf16(G0, G1, a.c2, ref, S0, W0, S1, W1);
+          if (v0 && !(W0 >= -3.0e38f && S0 <= 3.0e38f)) group_sums_bf16<true>(G0, a.c2, ref, S0, W0);
+          if (v1 && !(W1 >= -3.0e38f && S1 <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S1, W1);
+          if (new_top) {
+            const bool top0 = mg0 == mg;
+            lane_new_top(A, mg, top0 ? j0 : j1, top0 ? S0 : S1, top0 ? W0 : W1, a.c2);
+            const bool rest = top0 ? v1 : v0;
+            if (rest) {
+              A.Sr += top0 ? S1 : S0;
+              A.Wr += top0 ? W1 : W0;
+            }
+          } else {
+            if (v0) {
+              A.Sr += S0;
+              A.Wr += W0;
+            }
+            if (v1) {
+              A.Sr += S1;
+              A.Wr += W1;
+            }
+          }
+          if (sampling) {
+            if (v0) lane_race(A, S0, x0, j0);
+            if (v1) lane_race(A, S1, x1, j1);
+          }
+          continue;
+        }
+      }
+      // Any other tile: its description first.
+      const TileMeta m = meta[st];
+      const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
       const bool any = sub * Sh::kSubGroups < m.cnt;  // warp-uniform
       const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
       const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
@@ -959,58 +1020,6 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
         }
         if (sampling) lane_race(A, Z, x, j);
       };
-      if (DT == kBF16 && fast && any) {
-        // both groups into registers, then the stage goes back to the
-        // producer; the row change (which may wait for a row slot) comes
-        // after the release
-        uint32_t G0[32], G1[32];
-        load_group_bf16(sbase + (size_t)(has0 ? gl0 : 0) * 128, rot, G0);
-        load_group_bf16(sbase + (size_t)(has1 ? gl1 : has0 ? gl0 : 0) * 128, rot, G1);
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[st]);
-        if (!enter_row(m)) {
-          fail = true;
-          break;
-        }
-        // Both groups against one reference, the larger of the lane's
-        // maximum and theirs: a group raising it becomes the top group (the
-        // first on equal maxima), the other joins the rest; then the race,
-        // group 0 first.
-        const float mg0 = has0 ? group_max_bf16(G0) : -INFINITY;
-        const float mg1 = has1 ? group_max_bf16(G1) : -INFINITY;
-        const bool v0 = mg0 > -INFINITY, v1 = mg1 > -INFINITY;  // not every logit -inf
-        if (!(v0 || v1)) continue;
-        const float mg = fmaxf(mg0, mg1);
-        const bool new_top = mg > A.M;
-        const float ref = new_top ? mg : A.M;
-        float S0, W0, S1, W1;
-        group_sums2_bf16(G0, G1, a.c2, ref, S0, W0, S1, W1);
-        if (v0 && !(W0 >= -3.0e38f && S0 <= 3.0e38f)) group_sums_bf16<true>(G0, a.c2, ref, S0, W0);
-        if (v1 && !(W1 >= -3.0e38f && S1 <= 3.0e38f)) group_sums_bf16<true>(G1, a.c2, ref, S1, W1);
-        if (new_top) {
-          const bool top0 = mg0 == mg;
-          lane_new_top(A, mg, top0 ? j0 : j1, top0 ? S0 : S1, top0 ? W0 : W1, a.c2);
-          const bool rest = top0 ? v1 : v0;
-          if (rest) {
-            A.Sr += top0 ? S1 : S0;
-            A.Wr += top0 ? W1 : W0;
-          }
-        } else {
-          if (v0) {
-            A.Sr += S0;
-            A.Wr += W0;
-          }
-          if (v1) {
-            A.Sr += S1;
-            A.Wr += W1;
-          }
-        }
-        if (sampling) {
-          if (v0) lane_race(A, S0, x0, j0);
-          if (v1) lane_race(A, S1, x1, j1);
-        }
-        continue;
-      }
       if (!enter_row(m)) {
         fail = true;
         break;
