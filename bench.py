@@ -86,6 +86,13 @@ def peaks():
         return FALLBACK_HBM_GBS, "fallback"
 
 
+def peak_label(kind, key, fallback):
+    """Where a roofline peak came from."""
+    if kind == "measured":
+        return f"measured: MEASURED_PEAKS.json {key}"
+    return f"fallback: {fallback}, an earlier B200 measurement (no MEASURED_PEAKS.json)"
+
+
 def tensor_peak():
     """Dense bf16 tensor peak (TFLOP/s): the measured burst figure, else the
     pool's fallback."""
@@ -161,7 +168,8 @@ def run_lmhead_config(E, synth, dev, B, d, barrier, max_over_ranks):
         "roofline": {"bound": "tensor", "achieved": tfl, "peak": peak, "unit": "TFLOP/s",
                      "frac": tfl / peak, "kernel": "ebk::lmhead_kernel<true>",
                      "flop_per_step": flop,
-                     "peak_source": f"{kind} MEASURED_PEAKS.json bf16_tflops (cuBLAS burst)"},
+                     "peak_source": peak_label(kind, "bf16_tflops (cuBLAS burst)",
+                                               f"{FALLBACK_BF16_TFLOPS:.0f} TFLOP/s")},
     }
 
 
@@ -437,7 +445,7 @@ def roofline_of(kernel, launches, bytes_total, region_ms, peak, peak_kind):
             "algorithmic_bytes": bytes_launch,
             "timing": "CUDA events around graph replays on the launching stream; "
                       "region time / step-kernel launches",
-            "peak_source": f"{peak_kind} MEASURED_PEAKS.json hbm_gbs (copy)"}
+            "peak_source": peak_label(peak_kind, "hbm_gbs (copy)", f"{FALLBACK_HBM_GBS:.0f} GB/s")}
 
 
 LMHEAD_D = 2560  # hidden size of the LM-head configs (the pages give none)
