@@ -191,8 +191,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
 // mbar_wait, except that a limit shorter than kSuspendHintNs is kept with
 // tests that never suspend and the clock read after each: such a limit runs
 // out whenever the phase is not complete at the first test.
-__device__ __noinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                             const int* abort) {
+static __device__ __noinline__ bool mbar_wait_timed(uint64_t* bar, uint32_t parity,
+                                                    uint64_t limit_ns, const int* abort) {
   if (limit_ns >= kSuspendHintNs) return mbar_wait(bar, parity, limit_ns, abort);
   const uint64_t t0 = global_ns();
   for (;;) {

@@ -20,13 +20,19 @@
 //     stage before any arithmetic, so the ring refills while it computes.
 //     When a warp leaves a row it merges its lanes and deposits one record
 //     per row of the CTA's range into a shared-memory slot;
-//   - the finisher warp merges the twelve deposits of each row into the
-//     CTA's part of the row, made final (the exact top group and the element
-//     drawn in its best Gumbel group).  A row spread over several CTAs
-//     exchanges these records through global memory: each CTA writes its
-//     record and counts itself in the row's counter (or sees that the others
-//     are done already); the last one combines them (in CTA order) and
-//     writes the position's entropy, max probability, argmax and draw.
+//   - two finisher warps (alternating rows) merge the twelve deposits of
+//     each row into the CTA's part of the row, made final (the exact top
+//     group and the element drawn in its best Gumbel group).  A row spread
+//     over several CTAs exchanges these records through global memory: each
+//     CTA writes its record and counts itself in the row's counter (or sees
+//     that the others are done already); the last one combines them (in CTA
+//     order) and writes the position's entropy, max probability, argmax and
+//     draw.
+// The roles hand work to one another through mbarrier phases, in which a
+// waiting thread is suspended rather than polling shared memory: the
+// start-up publication (ready), a tile's description (described), a
+// stage's copy and header (full), its release (empty) and a row's twelve
+// deposits (the row slot's barrier).
 // The CTA that finishes a canvas's last position then runs that canvas's
 // decisions with all its threads (eb_finish.cuh), once every CTA of the
 // grid has read the stop flags.  Consecutive steps' kernels are chained by
@@ -78,7 +84,7 @@ __host__ __device__ constexpr int stream_threads(int dt) {
 
 struct StreamCtrl {
   int abort;
-  int issued;  // tiles whose bulk copy has been issued
+  int issued;  // tiles whose bulk copy has been issued (the exit drain's count)
   int n_sub;   // sub-tiles of this CTA's range
   int words_arrived;  // tiles whose second (header) arrival was made
   int n_epi;          // canvases whose decisions this CTA runs
