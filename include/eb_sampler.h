@@ -318,8 +318,12 @@ int eb_sampler_set_split_event(eb_sampler_t* h, void* event);
    A wait that runs out sets EB_STATUS_TIMEOUT, ends the step's stream pass
    early (the step's outputs are then not valid) and leaves the device
    usable; the wait for copies still in flight when the kernel exits keeps
-   its own 2 s limit.  Tests use a tiny limit to drive that error path
-   without a fault.  After a timeout, start the canvases again with
+   its own 2 s limit.  A waiting thread is suspended until the awaited
+   event happens, so the limit bounds waits for events that do not happen;
+   below 20 us the start-up wait (every role waiting for the first copy to
+   be issued) tests without suspending, so a tiny limit runs out there.
+   Tests use a tiny limit to drive that error path without a fault.  The
+   LM-head step's waits use the same limit.  After a timeout, start the canvases again with
    eb_sampler_init_canvas (which also clears the row counters a cut-short
    step may leave).  No counterpart in the method. */
 int eb_sampler_set_wait_limit(eb_sampler_t* h, uint64_t limit_ns);
