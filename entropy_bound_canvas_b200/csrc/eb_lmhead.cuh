@@ -7,9 +7,9 @@
 // model card's summary table: a vocabulary of about 262K).
 //
 // One CTA per SM, six warps:
-//   warp 0  producer: TMA (cp.async.bulk.tensor, 128-byte swizzle, no
-//           multicast) of a 128 x 64 tile of h and a 256 x 64 tile of W per
-//           stage, into a ring of kLmStages stages;
+//   warp 0  producer: TMA (cp.async.bulk.tensor, 128-byte swizzle, each
+//           CTA loading for itself) of a 128 x 64 tile of h and a 256 x 64
+//           tile of W per stage, into a ring of kLmStages stages;
 //   warp 1  MMA issuer: one elected thread issues tcgen05.mma (kind::f16,
 //           bf16 in, fp32 accumulate, M = 128, N = 256, K = 16 per
 //           instruction) into one of two TMEM accumulators (2 x 256 columns)
