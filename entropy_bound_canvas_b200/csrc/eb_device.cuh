@@ -103,8 +103,8 @@ __device__ __forceinline__ uint32_t uniform_token(uint32_t x, uint32_t V) { retu
 
 // ---------------------------------------------------------------------------
 // mbarrier + 1-D bulk copy (cp.async.bulk, the TMA engine without a tensor
-// map).  No multicast anywhere: every copy reads this GPU's own memory into
-// this CTA's shared memory.
+// map).  Every copy reads this GPU's own memory into the issuing CTA's own
+// shared memory and nowhere else.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));

@@ -10,7 +10,7 @@
 //   - the copy producer (one lane) walks the range in tiles of up to
 //     kStageGroups groups that never straddle a row, writes each tile's
 //     description and copies it into a kStages-deep ring with one 1-D bulk
-//     copy (the TMA engine, no multicast, L2 evict-first);
+//     copy (the TMA engine, into this CTA only, L2 evict-first);
 //   - the word producer computes the group-stream Philox words of an open
 //     position's tiles;
 //   - twelve consumer warps take the tiles' 64-group sub-tiles round-robin
