@@ -995,13 +995,15 @@ __global__ void __launch_bounds__(StreamShape<DT>::kThreads, 1) stream_kernel(co
           continue;
         }
       }
-      // Any other tile: its description first.
+      // Any other tile (fp32 logits; bf16 rows off 16-byte boundaries or a
+      // row's partial last group): its description first.
       const TileMeta m = meta[st];
       const unsigned char* sbase = ring + (size_t)st * Sh::kStageStride + m.delta;
       const bool any = sub * Sh::kSubGroups < m.cnt;  // warp-uniform
       const bool has0 = gl0 < m.cnt, has1 = gl1 < m.cnt;
       const int j0 = m.j0 + gl0, j1 = m.j0 + gl1;
-      // whole 16-byte-aligned groups in the whole tile: the vector path
+      // fp32: whole 16-byte-aligned groups in the whole tile take the vector
+      // path; every other group is read element by element
       const bool fast = m.whole != 0;
       uint32_t x0 = 0, x1 = 0;
       if (m.sampling) {
